@@ -1,0 +1,200 @@
+"""Exact memory-efficient attention for B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libmea_attn.so`` (include/mea_attn.h).
+The functions below carry the C names and only marshal arguments: tensor data
+pointers, sizes and the current CUDA stream.  Every step of the computation
+runs in the library's CUDA kernels; there is no CPU or PyTorch fallback, and
+loading fails loudly if the library has not been built.  PyTorch is used only
+to own device memory and streams.
+
+    o, lse = attention_forward(q, k, v)                 # allocates o, lse
+    dq, dk, dv = attention_backward(q, k, v, o, lse, do)  # allocates grads + workspace
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = [
+    "MeaError", "load_library", "library_path",
+    "MEA_OK", "MEA_ERR_INVALID_ARG", "MEA_ERR_UNSUPPORTED", "MEA_ERR_MISALIGNED", "MEA_ERR_WORKSPACE",
+    "MEA_ERR_CUDA", "MEA_ERR_TIMEOUT", "MEA_DTYPE_F32", "MEA_DTYPE_BF16",
+    "mea_attn_fwd", "mea_attn_bwd", "mea_attn_bwd_workspace_size", "mea_last_device_error",
+    "mea_status_string", "mea_last_error_message", "mea_version", "attention_forward", "attention_backward",
+]
+
+MEA_OK = 0
+MEA_ERR_INVALID_ARG = 1
+MEA_ERR_UNSUPPORTED = 2
+MEA_ERR_MISALIGNED = 3
+MEA_ERR_WORKSPACE = 4
+MEA_ERR_CUDA = 5
+MEA_ERR_TIMEOUT = 6
+
+MEA_DTYPE_F32 = 0
+MEA_DTYPE_BF16 = 1
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+
+
+def library_path() -> str:
+    return os.path.join(_PKG_DIR, "libmea_attn.so")
+
+
+class MeaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        detail = mea_last_error_message()
+        super().__init__(f"{where}: {mea_status_string(status)} (status {status})"
+                         + (f" [{detail}]" if detail else ""))
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libmea_attn.so from the package directory (raises if it is missing)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m exact_memory_efficient_b200.build` "
+            "(there is no fallback implementation)")
+    lib = ctypes.CDLL(path)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.mea_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+    lib.mea_attn_fwd.restype = i
+    lib.mea_attn_bwd_workspace_size.argtypes = [i, i, i, i, i, i, ctypes.POINTER(sz)]
+    lib.mea_attn_bwd_workspace_size.restype = i
+    lib.mea_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
+    lib.mea_attn_bwd.restype = i
+    lib.mea_last_device_error.argtypes = [vp]
+    lib.mea_last_device_error.restype = i
+    lib.mea_status_string.argtypes = [i]
+    lib.mea_status_string.restype = ctypes.c_char_p
+    lib.mea_last_error_message.argtypes = []
+    lib.mea_last_error_message.restype = ctypes.c_char_p
+    lib.mea_version.argtypes = []
+    lib.mea_version.restype = i
+    _LIB = lib
+    return lib
+
+
+def mea_status_string(status: int) -> str:
+    return load_library().mea_status_string(int(status)).decode()
+
+
+def mea_last_error_message() -> str:
+    return load_library().mea_last_error_message().decode()
+
+
+def mea_version() -> int:
+    return int(load_library().mea_version())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return MEA_DTYPE_F32
+    if t.dtype == torch.bfloat16:
+        return MEA_DTYPE_BF16
+    raise MeaError(MEA_ERR_UNSUPPORTED, f"dtype {t.dtype}")
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(status: int, where: str) -> None:
+    if status != MEA_OK:
+        raise MeaError(status, where)
+
+
+def _bhnd(t: torch.Tensor, name: str):
+    if t.dim() != 4:
+        raise MeaError(MEA_ERR_INVALID_ARG, f"{name} must be [B, H, N, D]")
+    if not t.is_contiguous():
+        raise MeaError(MEA_ERR_INVALID_ARG, f"{name} must be contiguous")
+    if not t.is_cuda:
+        raise MeaError(MEA_ERR_INVALID_ARG, f"{name} must be a CUDA tensor")
+    return t.shape
+
+
+def mea_attn_fwd(q, k, v, o, lse, scale: float, stream=None) -> None:
+    """C ``mea_attn_fwd``: writes o [B,H,Nq,D] and lse [B,H,Nq] (fp32) on the stream."""
+    B, H, Nq, D = _bhnd(q, "q")
+    Bk, Hk, Nk, Dk = _bhnd(k, "k")
+    if (Bk, Hk, Dk) != (B, H, D) or tuple(v.shape) != tuple(k.shape) or tuple(o.shape) != tuple(q.shape):
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_fwd: shape mismatch")
+    if tuple(lse.shape) != (B, H, Nq) or lse.dtype != torch.float32:
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_fwd: lse must be fp32 [B, H, Nq]")
+    if not (q.dtype == k.dtype == v.dtype == o.dtype):
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_fwd: dtype mismatch")
+    st = load_library().mea_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, D,
+                                      float(scale), _dtype_code(q), _stream_handle(stream))
+    _check(st, "mea_attn_fwd")
+
+
+def mea_attn_bwd_workspace_size(B: int, H: int, Nq: int, Nk: int, D: int, dtype=torch.bfloat16) -> int:
+    out = ctypes.c_size_t(0)
+    code = MEA_DTYPE_BF16 if dtype == torch.bfloat16 else MEA_DTYPE_F32
+    st = load_library().mea_attn_bwd_workspace_size(B, H, Nq, Nk, D, code, ctypes.byref(out))
+    _check(st, "mea_attn_bwd_workspace_size")
+    return int(out.value)
+
+
+def mea_attn_bwd(q, k, v, o, lse, do, dq, dk, dv, scale: float, workspace, stream=None) -> None:
+    """C ``mea_attn_bwd``: writes dq, dk, dv; ``workspace`` is a uint8 CUDA tensor."""
+    B, H, Nq, D = _bhnd(q, "q")
+    _, _, Nk, _ = _bhnd(k, "k")
+    for name, t, shape in (("o", o, q.shape), ("do", do, q.shape), ("dq", dq, q.shape), ("v", v, k.shape),
+                           ("dk", dk, k.shape), ("dv", dv, k.shape)):
+        if tuple(t.shape) != tuple(shape) or t.dtype != q.dtype:
+            raise MeaError(MEA_ERR_INVALID_ARG, f"mea_attn_bwd: {name} shape/dtype mismatch")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load_library().mea_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+                                      _ptr(dv), B, H, Nq, Nk, D, float(scale), _dtype_code(q), _ptr(workspace),
+                                      ws_bytes, _stream_handle(stream))
+    _check(st, "mea_attn_bwd")
+
+
+def mea_last_device_error(stream=None) -> int:
+    """C ``mea_last_device_error``: synchronises the stream and returns (and clears) the device flag."""
+    return int(load_library().mea_last_device_error(_stream_handle(stream)))
+
+
+# ---------------------------------------------------------------- helpers
+
+def attention_forward(q, k, v, scale: float | None = None, stream=None):
+    """Allocate (o, lse) with torch and run ``mea_attn_fwd``."""
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    mea_attn_fwd(q, k, v, o, lse, scale, stream)
+    return o, lse
+
+
+def attention_backward(q, k, v, o, lse, do, scale: float | None = None, workspace=None, stream=None):
+    """Allocate (dq, dk, dv) and, unless given, the workspace; run ``mea_attn_bwd``."""
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    B, H, Nq, D = q.shape
+    Nk = k.shape[2]
+    if workspace is None:
+        workspace = torch.empty(mea_attn_bwd_workspace_size(B, H, Nq, Nk, D, q.dtype), dtype=torch.uint8,
+                                device=q.device)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    mea_attn_bwd(q, k, v, o, lse, do, dq, dk, dv, scale, workspace, stream)
+    return dq, dk, dv

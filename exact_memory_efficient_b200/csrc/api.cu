@@ -1,0 +1,270 @@
+// api.cu -- the C ABI declared in include/mea_attn.h: argument validation,
+// dispatch, TMA tensor-map encoding and launches on the caller's stream.
+// Nothing here allocates, frees or synchronises on the fwd/bwd paths.
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "mea_attn.h"
+
+namespace mea {
+__device__ unsigned int g_device_error = 0;
+}
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// Text of the most recent failure on this host thread (mea_last_error_message).
+thread_local char g_err_msg[256] = "";
+
+mea_status_t fail(mea_status_t st, const char* where, const char* detail) {
+    std::snprintf(g_err_msg, sizeof(g_err_msg), "%s: %s", where, detail ? detail : "");
+    return st;
+}
+mea_status_t fail_cuda(const char* where, cudaError_t e) {
+    return fail(MEA_ERR_CUDA, where, cudaGetErrorString(e));
+}
+
+struct DeviceInfo {
+    bool init = false;
+    bool sm100 = false;
+    int sm_count = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+mea_status_t device_info(DeviceInfo** out) {
+    int dev = 0;
+    cudaError_t ce = cudaGetDevice(&dev);
+    if (ce != cudaSuccess) return fail_cuda("cudaGetDevice", ce);
+    if (dev < 0 || dev >= kMaxDevices) return MEA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.init) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return fail(MEA_ERR_CUDA, "cudaDeviceGetAttribute", "failed");
+        d.sm100 = (major == 10 && minor == 0);
+        d.sm_count = sms;
+        d.init = true;
+    }
+    if (g_encode == nullptr) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return fail(MEA_ERR_CUDA, "cudaGetDriverEntryPoint", "cuTensorMapEncodeTiled unavailable");
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    if (!d.sm100) return fail(MEA_ERR_UNSUPPORTED, "device", "compute capability 10.0 (sm_100a) required");
+    *out = &d;
+    return MEA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// 3-D bf16 map over [BH][N][D]: dims {D, N, BH}, box {64, 128, 1}, 128-byte swizzle,
+// out-of-range rows read as zero.
+mea_status_t make_map(CUtensorMap* m, const void* base, int BH, int N, int D) {
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * D * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        char buf[64];
+        std::snprintf(buf, sizeof(buf), "CUresult %d", (int)r);
+        return fail(MEA_ERR_CUDA, "cuTensorMapEncodeTiled", buf);
+    }
+    return MEA_OK;
+}
+
+mea_status_t common_checks(int B, int H, int Nq, int Nk, int D, float scale, mea_dtype_t dtype) {
+    if (dtype != MEA_DTYPE_F32 && dtype != MEA_DTYPE_BF16) return MEA_ERR_INVALID_ARG;
+    if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || D <= 0) return MEA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return MEA_ERR_INVALID_ARG;
+    if ((long long)B * H > 0x7fffffffLL) return MEA_ERR_INVALID_ARG;
+    const long long maxn = Nq > Nk ? Nq : Nk;
+    if ((long long)B * H * maxn * D >= (1LL << 40)) return MEA_ERR_INVALID_ARG;
+    if (dtype == MEA_DTYPE_BF16 && D != 64 && D != 128) return MEA_ERR_UNSUPPORTED;
+    if (dtype == MEA_DTYPE_F32 && (D % 32 != 0 || D > 128)) return MEA_ERR_UNSUPPORTED;
+    return MEA_OK;
+}
+
+mea_status_t cuda_status(cudaError_t e, const char* where) {
+    return e == cudaSuccess ? MEA_OK : fail_cuda(where, e);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mea_status_string(mea_status_t s) {
+    switch (s) {
+        case MEA_OK: return "MEA_OK";
+        case MEA_ERR_INVALID_ARG: return "MEA_ERR_INVALID_ARG: invalid argument";
+        case MEA_ERR_UNSUPPORTED: return "MEA_ERR_UNSUPPORTED: unsupported dtype, head dim, direction or device";
+        case MEA_ERR_MISALIGNED: return "MEA_ERR_MISALIGNED: pointer misaligned";
+        case MEA_ERR_WORKSPACE: return "MEA_ERR_WORKSPACE: workspace missing or too small";
+        case MEA_ERR_CUDA: return "MEA_ERR_CUDA: CUDA call or launch failed";
+        case MEA_ERR_TIMEOUT: return "MEA_ERR_TIMEOUT: a device-side bounded wait expired";
+    }
+    return "MEA_ERR_UNKNOWN";
+}
+
+int mea_version(void) { return 100; }
+
+const char* mea_last_error_message(void) { return g_err_msg; }
+
+mea_status_t mea_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                          int Nk, int D, float scale, mea_dtype_t dtype, void* stream) {
+    mea_status_t st = common_checks(B, H, Nq, Nk, D, scale, dtype);
+    if (st != MEA_OK) return st;
+    const long long rows = (long long)B * H * Nq;
+    if (rows == 0) return MEA_OK;
+    if (Nk == 0) return MEA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !o || !lse) return MEA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse)) return MEA_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    if ((st = device_info(&dev)) != MEA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int BH = B * H;
+
+    if (dtype == MEA_DTYPE_F32) {
+        mea::F32FwdArgs a;
+        a.q = static_cast<const float*>(q);
+        a.k = static_cast<const float*>(k);
+        a.v = static_cast<const float*>(v);
+        a.o = static_cast<float*>(o);
+        a.lse = lse;
+        a.BH = BH;
+        a.Nq = Nq;
+        a.Nk = Nk;
+        a.D = D;
+        a.scale = scale;
+        if (Nq >= 8) { a.rows_per_cta = 8; a.warps_per_row = 1; }
+        else if (Nq >= 4) { a.rows_per_cta = 4; a.warps_per_row = 2; }
+        else if (Nq >= 2) { a.rows_per_cta = 2; a.warps_per_row = 4; }
+        else { a.rows_per_cta = 1; a.warps_per_row = 8; }
+        const long long base = (long long)BH * ((Nq + a.rows_per_cta - 1) / a.rows_per_cta);
+        const long long target = 2LL * dev->sm_count;
+        int chunks = 1;
+        while (chunks < 16 && base * chunks < target &&
+               (long long)Nk / (2 * chunks) >= 2LL * 32 * a.warps_per_row)
+            chunks *= 2;
+        a.chunks = chunks;
+        const long long per = (Nk + chunks - 1) / chunks;
+        a.chunk_len = (int)round_up((size_t)per, 32);
+        if ((long long)((Nq + a.rows_per_cta - 1) / a.rows_per_cta) > 65535 || BH > 65535)
+            return MEA_ERR_UNSUPPORTED;
+        return cuda_status(mea::launch_fwd_f32(a, s), "fwd_f32 launch");
+    }
+
+    mea::Bf16FwdArgs a;
+    if ((st = make_map(&a.tm_q, q, BH, Nq, D)) != MEA_OK) return st;
+    if ((st = make_map(&a.tm_k, k, BH, Nk, D)) != MEA_OK) return st;
+    if ((st = make_map(&a.tm_v, v, BH, Nk, D)) != MEA_OK) return st;
+    a.o = static_cast<uint16_t*>(o);
+    a.lse = lse;
+    a.BH = BH;
+    a.Nq = Nq;
+    a.Nk = Nk;
+    a.D = D;
+    a.scale = scale;
+    if (BH > 65535) return MEA_ERR_UNSUPPORTED;
+    return cuda_status(mea::launch_fwd_bf16(a, s), "fwd_bf16 launch");
+}
+
+mea_status_t mea_attn_bwd_workspace_size(int B, int H, int Nq, int Nk, int D, mea_dtype_t dtype, size_t* bytes) {
+    if (bytes == nullptr) return MEA_ERR_INVALID_ARG;
+    mea_status_t st = common_checks(B, H, Nq, Nk, D, 1.0f, dtype);
+    if (st != MEA_OK) return st;
+    if (dtype != MEA_DTYPE_BF16) return MEA_ERR_UNSUPPORTED;
+    const size_t rows = (size_t)B * H * Nq;
+    *bytes = round_up(rows * D * sizeof(float), 256) + round_up(rows * sizeof(float), 256);
+    return MEA_OK;
+}
+
+mea_status_t mea_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                          const void* dO, void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int D,
+                          float scale, mea_dtype_t dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    mea_status_t st = common_checks(B, H, Nq, Nk, D, scale, dtype);
+    if (st != MEA_OK) return st;
+    if (dtype != MEA_DTYPE_BF16) return MEA_ERR_UNSUPPORTED;
+    const int BH = B * H;
+    if (BH == 0) return MEA_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (Nq == 0) {
+        if (Nk == 0) return MEA_OK;
+        if (!dk || !dv) return MEA_ERR_INVALID_ARG;
+        if (!aligned16(dk) || !aligned16(dv)) return MEA_ERR_MISALIGNED;
+        const size_t n = (size_t)BH * Nk * D * 2;
+        cudaError_t e = cudaMemsetAsync(dk, 0, n, s);
+        if (e != cudaSuccess) return fail_cuda("cudaMemsetAsync", e);
+        return cuda_status(cudaMemsetAsync(dv, 0, n, s), "cudaMemsetAsync");
+    }
+    if (Nk == 0) return MEA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return MEA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv) || !aligned4(lse))
+        return MEA_ERR_MISALIGNED;
+    size_t need = 0;
+    if ((st = mea_attn_bwd_workspace_size(B, H, Nq, Nk, D, dtype, &need)) != MEA_OK) return st;
+    if (workspace == nullptr || workspace_bytes < need) return MEA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MEA_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    if ((st = device_info(&dev)) != MEA_OK) return st;
+    if (BH > 65535) return MEA_ERR_UNSUPPORTED;
+
+    mea::Bf16BwdArgs a;
+    if ((st = make_map(&a.tm_q, q, BH, Nq, D)) != MEA_OK) return st;
+    if ((st = make_map(&a.tm_k, k, BH, Nk, D)) != MEA_OK) return st;
+    if ((st = make_map(&a.tm_v, v, BH, Nk, D)) != MEA_OK) return st;
+    if ((st = make_map(&a.tm_do, dO, BH, Nq, D)) != MEA_OK) return st;
+    const size_t rows = (size_t)BH * Nq;
+    a.o = static_cast<const uint16_t*>(o);
+    a.dO = static_cast<const uint16_t*>(dO);
+    a.lse = lse;
+    a.dq = static_cast<uint16_t*>(dq);
+    a.dk = static_cast<uint16_t*>(dk);
+    a.dv = static_cast<uint16_t*>(dv);
+    a.dq_acc = static_cast<float*>(workspace);
+    a.delta = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round_up(rows * D * sizeof(float), 256));
+    a.BH = BH;
+    a.Nq = Nq;
+    a.Nk = Nk;
+    a.D = D;
+    a.scale = scale;
+    return cuda_status(mea::launch_bwd_bf16(a, s), "bwd_bf16 launch");
+}
+
+mea_status_t mea_last_device_error(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail_cuda("cudaStreamSynchronize", e);
+    unsigned int flag = 0;
+    if (cudaMemcpyFromSymbol(&flag, mea::g_device_error, sizeof(flag)) != cudaSuccess) return MEA_ERR_CUDA;
+    if (flag == 0) return MEA_OK;
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(mea::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return MEA_ERR_CUDA;
+    return (flag & 1u) ? MEA_ERR_TIMEOUT : MEA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,447 @@
+// bwd_bf16.cu -- bf16 backward on the 5th-generation tensor cores (sm_100a).
+//
+// Method: "Self-attention Does Not Need O(n^2) Memory" (English summary,
+// method bullet on differentiation): nothing of size n x n is stored by the
+// forward; the backward recomputes the probabilities block by block from the
+// saved per-row lse (checkpointing), P = exp(scale q k^T - lse).  The gradient
+// formulas are ordinary softmax calculus:
+//     dV = P^T dO,  dP = dO V^T,  D_i = sum_d dO_id O_id,  dS = P o (dP - D),
+//     dQ = scale dS K,  dK = scale dS^T Q.
+//
+// Three kernels on one stream:
+//   bwd_pre      D_i = sum_d dO_id O_id (fp32) and zeroes the fp32 dQ accumulator.
+//   bwd_main     one CTA per (batch*head, 128-key tile); loops over 128-query
+//                tiles.  Everything is computed transposed (keys on TMEM lanes):
+//                  S^T  = K Q_i^T          (smem x smem -> TMEM)
+//                  dP^T = V dO_i^T         (smem x smem -> TMEM)
+//                  dV  += P^T dO_i         (P^T from TMEM, bf16)
+//                  dK  += dS^T Q_i         (dS^T from TMEM, bf16)
+//                  dQ_i = dS K             (dS from smem, bf16) -> fp32 atomic adds
+//   bwd_dq_final dq = bf16(scale * dQacc).
+//
+// Roles in bwd_main (320 threads): warp 0 TMEM allocator and TMA producer (K, V
+// once; Q_i, dO_i through a 2-stage ring; no multicast), warp 1 MMA issuer,
+// warps 2-9 two compute groups of four warps; thread (warp w, lane) owns key
+// row 32*(w%4)+lane (the TMEM lane warp w can reach) and query half (w-2)/4 of
+// every tile.
+// TMEM: S^T [0,128)  dP^T [128,256)  dV [256,256+D)  dK [256+D, 256+2D)
+//       dQ: D=128 reuses the dP^T columns, D=64 uses [384,448).
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace mea {
+namespace {
+
+constexpr int kTile = 128;
+constexpr int kThreads = 320;
+constexpr int kComputeThreads = 256;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ------------------------------------------------------------------ pre
+
+// One warp per query row: delta = sum_d dO * O (fp32), and dq_acc row := 0.
+__global__ void bwd_pre_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dO,
+                               float* __restrict__ delta, float* __restrict__ dq_acc, long long rows, int D) {
+    const long long row = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x / 32);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const uint16_t* orow = o + row * D;
+    const uint16_t* drow = dO + row * D;
+    float acc = 0.f;
+    for (int d = 2 * lane; d < D; d += 64) {
+        const uint32_t ov = *reinterpret_cast<const uint32_t*>(orow + d);
+        const uint32_t dv = *reinterpret_cast<const uint32_t*>(drow + d);
+        acc = fmaf(__uint_as_float(ov << 16), __uint_as_float(dv << 16), acc);
+        acc = fmaf(__uint_as_float(ov & 0xffff0000u), __uint_as_float(dv & 0xffff0000u), acc);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) delta[row] = acc;
+    float4* z = reinterpret_cast<float4*>(dq_acc + row * D);
+    for (int c = lane; c < D / 4; c += 32) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// ------------------------------------------------------------- finalise
+
+__global__ void bwd_dq_final_kernel(const float* __restrict__ dq_acc, uint16_t* __restrict__ dq,
+                                    long long n4, float scale) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n4) return;
+    const float4 a = reinterpret_cast<const float4*>(dq_acc)[i];
+    uint2 r;
+    r.x = pack_bf16x2(a.x * scale, a.y * scale);
+    r.y = pack_bf16x2(a.z * scale, a.w * scale);
+    reinterpret_cast<uint2*>(dq)[i] = r;
+}
+
+// ----------------------------------------------------------------- main
+
+template <int D>
+struct BwdCfg {
+    static constexpr int kKVBytes = kTile * D * 2;      // one K (or V, Q, dO) tile
+    static constexpr int kStageBytes = 2 * kKVBytes;    // Q_i + dO_i
+    static constexpr int kStages = 2;
+    static constexpr int kDSBytes = kTile * kTile * 2;  // dS tile, bf16
+    static constexpr int kBoxBytes = 128 * 128;
+    static constexpr int offK = 0;
+    static constexpr int offV = kKVBytes;
+    static constexpr int offRing = 2 * kKVBytes;
+    static constexpr int offDS = offRing + kStages * kStageBytes;
+    static constexpr int offStats = offDS + kDSBytes;          // lse2[2][128], delta[2][128]
+    static constexpr int offBars = offStats + 4 * kTile * 4;
+    static constexpr int kSmemBytes = offBars + 256;
+    static constexpr bool kDqInDp = (D == 128);
+    static constexpr unsigned colS = 0, colDP = 128, colDV = 256, colDK = 256 + D;
+    static constexpr unsigned colDQ = kDqInDp ? 128u : 384u;
+};
+
+struct BwdBarriers {
+    uint64_t kv_full;
+    uint64_t q_full[2];
+    uint64_t q_empty[2];
+    uint64_t s_full, dp_full, dq_full;
+    uint64_t p_ready, ds_ready, dq_free;
+    uint64_t stats[2];
+    uint64_t final_done;
+    uint64_t drain;
+    unsigned tmem_base;
+    int abort_flag;
+};
+
+__device__ __forceinline__ uint64_t kmajor_desc(unsigned base, int kk) {
+    return make_sdesc_sw128(base + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+}
+__device__ __forceinline__ uint64_t mnmajor_desc(unsigned base, int kk) {
+    return make_sdesc_sw128(base + kk * 16 * 128, 128 * 128, 1024);
+}
+// bf16 A operand packed in TMEM by the two compute warpgroups: query half g
+// occupies columns [64 g, 64 g + 32) of its region.
+__device__ __forceinline__ unsigned packed_col(int kk) { return (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8; }
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const float* __restrict__ lse, const float* __restrict__ delta,
+                float* __restrict__ dq_acc, uint16_t* __restrict__ dk, uint16_t* __restrict__ dv,
+                int Nq, int Nk, float scale) {
+    using Cfg = BwdCfg<D>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    BwdBarriers* bars = reinterpret_cast<BwdBarriers*>(smem + Cfg::offBars);
+    float* s_lse2 = reinterpret_cast<float*>(smem + Cfg::offStats);          // [2][128]
+    float* s_delta = s_lse2 + 2 * kTile;                                      // [2][128]
+
+    const unsigned warp = warp_id();
+    const unsigned lane = lane_id();
+    const int bh = blockIdx.y;
+    const int n0 = blockIdx.x * kTile;      // first key of this CTA
+    const int n_q = (Nq + kTile - 1) / kTile;
+
+    if ((smem_u32(smem) & 1023u) != 0) {     // swizzle atoms need 1024-byte alignment
+        if (threadIdx.x == 0) flag_timeout();
+        return;
+    }
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->kv_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars->q_full[s], 1);
+            mbar_init(&bars->q_empty[s], 1);
+        }
+        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->dp_full, 1);
+        mbar_init(&bars->dq_full, 1);
+        mbar_init(&bars->p_ready, kComputeThreads);
+        mbar_init(&bars->ds_ready, kComputeThreads);
+        mbar_init(&bars->dq_free, kComputeThreads);
+        mbar_init(&bars->stats[0], kComputeThreads);
+        mbar_init(&bars->stats[1], kComputeThreads);
+        mbar_init(&bars->final_done, 1);
+        mbar_init(&bars->drain, 1);
+        bars->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&bars->tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const unsigned tmem = bars->tmem_base;
+    volatile int* abort_flag = &bars->abort_flag;
+    uint8_t* sK = smem + Cfg::offK;
+    uint8_t* sV = smem + Cfg::offV;
+    uint8_t* sRing = smem + Cfg::offRing;
+    uint8_t* sDS = smem + Cfg::offDS;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+            prefetch_tmap(&tm_do);
+            mbar_arrive_expect_tx(&bars->kv_full, 2 * Cfg::kKVBytes);
+            for (int b = 0; b < D / 64; ++b) {
+                tma_load_3d(sK + b * Cfg::kBoxBytes, &tm_k, &bars->kv_full, b * 64, n0, bh);
+                tma_load_3d(sV + b * Cfg::kBoxBytes, &tm_v, &bars->kv_full, b * 64, n0, bh);
+            }
+            int issued = 0;
+            for (int i = 0; i < n_q; ++i) {
+                const int st = i & 1;
+                if (i >= 2 && !mbar_wait(&bars->q_empty[st], ((i >> 1) - 1) & 1, abort_flag)) break;
+                uint8_t* dst = sRing + st * Cfg::kStageBytes;
+                mbar_arrive_expect_tx(&bars->q_full[st], Cfg::kStageBytes);
+                for (int b = 0; b < D / 64; ++b) {
+                    tma_load_3d(dst + b * Cfg::kBoxBytes, &tm_q, &bars->q_full[st], b * 64, i * kTile, bh);
+                    tma_load_3d(dst + Cfg::kKVBytes + b * Cfg::kBoxBytes, &tm_do, &bars->q_full[st], b * 64,
+                                i * kTile, bh);
+                }
+                issued = i + 1;
+            }
+            for (int i = (issued > 2 ? issued - 2 : 0); i < issued; ++i)
+                mbar_wait(&bars->q_full[i & 1], (i >> 1) & 1, nullptr);
+            mbar_wait(&bars->kv_full, 0, nullptr);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr unsigned idesc_t = make_idesc_bf16(128, 128, 0, 0);   // S^T, dP^T
+            constexpr unsigned idesc_g = make_idesc_bf16(128, D, 0, 1);     // dV, dK (A in TMEM)
+            constexpr unsigned idesc_q = make_idesc_bf16(128, D, 1, 1);     // dQ (A = dS, MN-major)
+            const unsigned aK = smem_u32(sK), aV = smem_u32(sV), aDS = smem_u32(sDS);
+            bool ok = mbar_wait(&bars->kv_full, 0, abort_flag);
+            for (int i = 0; ok && i < n_q; ++i) {
+                const int st = i & 1;
+                if (!(ok = mbar_wait(&bars->q_full[st], (i >> 1) & 1, abort_flag))) break;
+                tc_fence_after();
+                const unsigned aQ = smem_u32(sRing + st * Cfg::kStageBytes);
+                const unsigned aDO = aQ + Cfg::kKVBytes;
+                // S^T = K Q_i^T
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(tmem + Cfg::colS, kmajor_desc(aK, kk), kmajor_desc(aQ, kk), idesc_t, kk > 0);
+                mma_commit(&bars->s_full);
+                // dP^T = V dO_i^T  (D=128: dP columns held dQ_{i-1} until the compute warps freed them)
+                if (Cfg::kDqInDp && i > 0) {
+                    if (!(ok = mbar_wait(&bars->dq_free, (i - 1) & 1, abort_flag))) break;
+                    tc_fence_after();
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(tmem + Cfg::colDP, kmajor_desc(aV, kk), kmajor_desc(aDO, kk), idesc_t, kk > 0);
+                mma_commit(&bars->dp_full);
+                // dV += P^T dO_i
+                if (!(ok = mbar_wait(&bars->p_ready, i & 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    mma_ts(tmem + Cfg::colDV, tmem + Cfg::colS + packed_col(kk), mnmajor_desc(aDO, kk), idesc_g,
+                           (i > 0 || kk > 0));
+                // dK += dS^T Q_i ; dQ_i = dS K
+                if (!(ok = mbar_wait(&bars->ds_ready, i & 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    mma_ts(tmem + Cfg::colDK, tmem + Cfg::colDP + packed_col(kk), mnmajor_desc(aQ, kk), idesc_g,
+                           (i > 0 || kk > 0));
+                if (!Cfg::kDqInDp && i > 0) {
+                    if (!(ok = mbar_wait(&bars->dq_free, (i - 1) & 1, abort_flag))) break;
+                    tc_fence_after();
+                }
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    mma_ss(tmem + Cfg::colDQ, mnmajor_desc(aDS, kk), mnmajor_desc(aK, kk), idesc_q, kk > 0);
+                mma_commit(&bars->dq_full);
+                mma_commit(&bars->q_empty[st]);
+            }
+            if (ok) mma_commit(&bars->final_done);
+            mma_commit(&bars->drain);
+            mbar_wait(&bars->drain, 0, nullptr);
+        }
+    } else {
+        // ------------------------------------------------ compute warps
+        const int g = (warp - 2) >> 2;                 // query half of every tile
+        const unsigned sub = warp & 3;
+        const int kr = sub * 32 + lane;                // key row within the tile (TMEM lane)
+        const unsigned lane_off = (sub * 32u) << 16;
+        const int ctid = threadIdx.x - 64;             // 0..255
+        const float c_log2 = scale * kLog2e;
+        const bool key_ok = (n0 + kr) < Nk;
+        const float* lse_h = lse + (size_t)bh * Nq;
+        const float* delta_h = delta + (size_t)bh * Nq;
+        // stage lse2 / delta of tile 0
+        auto load_stats = [&](int i, float& lv, float& dvv) {
+            const int row = i * kTile + (ctid & 127);
+            lv = (row < Nq) ? lse_h[row] * kLog2e : INFINITY;
+            dvv = (row < Nq) ? delta_h[row] : 0.f;
+        };
+        float pre_l = 0.f, pre_d = 0.f;
+        load_stats(0, pre_l, pre_d);
+        bool ok = true;
+        for (int i = 0; i < n_q; ++i) {
+            const int slot = i & 1;
+            if (ctid < 128) s_lse2[slot * kTile + ctid] = pre_l;
+            else s_delta[slot * kTile + (ctid - 128)] = pre_d;
+            mbar_arrive(&bars->stats[slot]);
+            if (!(ok = mbar_wait(&bars->stats[slot], (i >> 1) & 1, abort_flag))) break;
+            if (i + 1 < n_q) load_stats(i + 1, pre_l, pre_d);
+            const float* l2 = s_lse2 + slot * kTile + 64 * g;
+            const float* dl = s_delta + slot * kTile + 64 * g;
+
+            // ---- P^T = exp2(scale*log2e * S^T - lse2), query half g
+            if (!(ok = mbar_wait(&bars->s_full, i & 1, abort_flag))) break;
+            tc_fence_after();
+            float p[64];
+            {
+                uint32_t sr[64];
+                tmem_ld32(tmem + lane_off + Cfg::colS + 64 * g, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                tmem_ld32(tmem + lane_off + Cfg::colS + 64 * g + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                    p[c] = key_ok ? ex2_approx(fmaf(__uint_as_float(sr[c]), c_log2, -l2[c])) : 0.f;
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
+                tmem_st32(tmem + lane_off + Cfg::colS + 64 * g, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars->p_ready);
+
+            // ---- dS^T = P^T o (dP^T - delta)
+            if (!(ok = mbar_wait(&bars->dp_full, i & 1, abort_flag))) break;
+            tc_fence_after();
+            {
+                uint32_t dr[64];
+                tmem_ld32(tmem + lane_off + Cfg::colDP + 64 * g, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+                tmem_ld32(tmem + lane_off + Cfg::colDP + 64 * g + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+                tmem_wait_ld();
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float d0 = p[2 * c] * (__uint_as_float(dr[2 * c]) - dl[2 * c]);
+                    const float d1 = p[2 * c + 1] * (__uint_as_float(dr[2 * c + 1]) - dl[2 * c + 1]);
+                    pk[c] = pack_bf16x2(d0, d1);
+                }
+                tmem_st32(tmem + lane_off + Cfg::colDP + 64 * g, pk);
+                // dS (queries x keys) for the dQ MMA: MN-major A operand, query block g,
+                // row = key, 16-byte chunk c of the 128-byte row swizzled by (key mod 8).
+                uint8_t* row = sDS + g * Cfg::kBoxBytes + kr * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const int pc = c ^ (kr & 7);
+                    *reinterpret_cast<uint4*>(row + pc * 16) =
+                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars->ds_ready);
+
+            // ---- dQacc[i] += dS K  (TMEM lanes are query rows here)
+            if (!(ok = mbar_wait(&bars->dq_full, i & 1, abort_flag))) break;
+            tc_fence_after();
+            {
+                const int q_row = i * kTile + kr;
+                float* dst = dq_acc + ((size_t)bh * Nq + q_row) * D + g * (D / 2);
+#pragma unroll
+                for (int c0 = 0; c0 < D / 2; c0 += 32) {
+                    uint32_t qv[32];
+                    tmem_ld32(tmem + lane_off + Cfg::colDQ + g * (D / 2) + c0, qv);
+                    tmem_wait_ld();
+                    if (q_row < Nq) {
+#pragma unroll
+                        for (int c = 0; c < 32; c += 4)
+                            red_add_v4(dst + c0 + c, __uint_as_float(qv[c]), __uint_as_float(qv[c + 1]),
+                                       __uint_as_float(qv[c + 2]), __uint_as_float(qv[c + 3]));
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&bars->dq_free);
+        }
+        // ---- epilogue: dV, dK (scaled) rows of this CTA's keys
+        if (ok && mbar_wait(&bars->final_done, 0, abort_flag)) {
+            tc_fence_after();
+            const int key = n0 + kr;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const unsigned col = (which == 0 ? Cfg::colDV : Cfg::colDK) + g * (D / 2);
+                const float mul = (which == 0) ? 1.f : scale;
+                uint16_t* dst = (which == 0 ? dv : dk) + ((size_t)bh * Nk + key) * D + g * (D / 2);
+#pragma unroll
+                for (int c0 = 0; c0 < D / 2; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_off + col + c0, r);
+                    tmem_wait_ld();
+                    if (key_ok) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int c = 0; c < 16; ++c)
+                            pk[c] = pack_bf16x2(__uint_as_float(r[2 * c]) * mul, __uint_as_float(r[2 * c + 1]) * mul);
+                        uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int D>
+cudaError_t launch_main(const Bf16BwdArgs& a, cudaStream_t stream) {
+    using Cfg = BwdCfg<D>;
+    static_assert(Cfg::kSmemBytes <= 232448, "shared memory budget");
+    auto kern = bwd_main_kernel<D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    dim3 grid((a.Nk + kTile - 1) / kTile, a.BH, 1);
+    kern<<<grid, kThreads, Cfg::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.lse, a.delta, a.dq_acc,
+                                                      a.dk, a.dv, a.Nq, a.Nk, a.scale);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_bf16(const Bf16BwdArgs& a, cudaStream_t stream) {
+    const long long rows = (long long)a.BH * a.Nq;
+    if (rows > 0) {
+        const int warps = 8;
+        const long long blocks = (rows + warps - 1) / warps;
+        bwd_pre_kernel<<<(unsigned)blocks, 32 * warps, 0, stream>>>(a.o, a.dO, a.delta, a.dq_acc, rows, a.D);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    cudaError_t e = (a.D == 64) ? launch_main<64>(a, stream) : (a.D == 128) ? launch_main<128>(a, stream)
+                                                                              : cudaErrorInvalidValue;
+    if (e != cudaSuccess) return e;
+    if (rows > 0) {
+        const long long n4 = rows * a.D / 4;
+        const int tpb = 256;
+        bwd_dq_final_kernel<<<(unsigned)((n4 + tpb - 1) / tpb), tpb, 0, stream>>>(a.dq_acc, a.dq, n4, a.scale);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+
+}  // namespace mea

@@ -1,0 +1,55 @@
+// kernels.h -- internal launch interface between the C ABI (api.cu) and the
+// kernels.  Not installed; the public interface is include/mea_attn.h.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace mea {
+
+// fp32 SIMT forward (fwd_f32.cu).
+struct F32FwdArgs {
+    const float* q;
+    const float* k;
+    const float* v;
+    float* o;
+    float* lse;
+    int BH, Nq, Nk, D;
+    float scale;
+    int rows_per_cta;   // query rows per CTA (one row per group of warps_per_row warps)
+    int warps_per_row;  // warps sharing one row's keys inside a CTA
+    int chunks;         // CTAs per cluster splitting the keys (1..16)
+    int chunk_len;      // keys per chunk (multiple of 32)
+};
+cudaError_t launch_fwd_f32(const F32FwdArgs& a, cudaStream_t stream);
+
+// bf16 tcgen05 forward (fwd_bf16.cu).  Tensor maps are 3-D {D, N, B*H} bf16,
+// 128-byte swizzle, box {64, 128, 1}.
+struct Bf16FwdArgs {
+    CUtensorMap tm_q, tm_k, tm_v;
+    uint16_t* o;  // bf16 bits
+    float* lse;
+    int BH, Nq, Nk, D;
+    float scale;
+};
+cudaError_t launch_fwd_bf16(const Bf16FwdArgs& a, cudaStream_t stream);
+
+// bf16 backward (bwd_bf16.cu).
+struct Bf16BwdArgs {
+    CUtensorMap tm_q, tm_k, tm_v, tm_do;
+    const uint16_t* o;
+    const uint16_t* dO;
+    const float* lse;
+    uint16_t* dq;
+    uint16_t* dk;
+    uint16_t* dv;
+    float* dq_acc;  // workspace [BH, Nq, D] fp32
+    float* delta;   // workspace [BH, Nq] fp32: sum_d dO * O
+    int BH, Nq, Nk, D;
+    float scale;
+};
+cudaError_t launch_bwd_bf16(const Bf16BwdArgs& a, cudaStream_t stream);
+
+}  // namespace mea

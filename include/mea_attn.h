@@ -1,0 +1,149 @@
+/*
+ * mea_attn.h -- C ABI of the exact memory-efficient attention library
+ * (libmea_attn.so, sm_100a).
+ *
+ * The operation is exact softmax attention for every (batch, head):
+ *
+ *     O = softmax(scale * Q K^T) V,      lse_i = ln sum_j exp(scale * q_i . k_j)
+ *
+ * as defined in "Fast and memory-efficient exact attention" (section on the
+ * mathematical form: softmax(QK^T / sqrt(d_k)) V) and computed the way
+ * "Self-attention Does Not Need O(n^2) Memory" describes (English summary,
+ * method bullets): keys and values are consumed block by block, each query row
+ * keeps a running maximum score, a running sum of exponentials and a rescaled
+ * weighted-value accumulator, and normalisation happens once at the end, so
+ * the n x n score matrix is never stored.  The backward pass recomputes the
+ * probabilities from lse instead of storing them (the same page's bullet on
+ * differentiation by checkpointing).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are contiguous row-major [B, H, N, D] ("BHND"); d_v = d.
+ *    q, o, dO, dq: [B, H, Nq, D];  k, v, dk, dv: [B, H, Nk, D];
+ *    lse: [B, H, Nq] fp32 (natural log of the scaled scores' exp-sum).
+ *  - Every pointer is caller-owned DEVICE memory.  The library never
+ *    allocates, frees or synchronises inside fwd/bwd; scratch memory for the
+ *    backward pass is the caller's `workspace`.
+ *  - Tensor pointers (q, k, v, o, dO, dq, dk, dv, workspace) must be 16-byte
+ *    aligned; lse must be 4-byte aligned.
+ *  - `stream` is a cudaStream_t (CUstream) passed as void*; NULL means the
+ *    legacy default stream.  Work is enqueued asynchronously; a returned
+ *    MEA_OK means the arguments were valid and the launches were accepted.
+ *  - Arguments are validated on the host before anything is launched; an
+ *    invalid call returns an error status and leaves all outputs untouched.
+ *    The library never aborts the process.
+ *  - Device-side failures that do not stop a launch (a bounded wait that
+ *    expired) set a per-device flag that mea_last_device_error() reports.
+ *
+ * Supported set
+ *  - MEA_DTYPE_BF16: forward and backward, D in {64, 128}; inputs/outputs bf16,
+ *    accumulation fp32 (tcgen05 tensor cores).
+ *  - MEA_DTYPE_F32: forward only, D in {32, 64, 96, 128}; fp32 throughout.
+ *  - Any Nq >= 0 and Nk >= 1; partial tiles are masked.  No mask, no dropout.
+ *  - B*H <= 2^31-1 and B*H*max(Nq,Nk)*D < 2^40 elements.
+ */
+#ifndef MEA_ATTN_H
+#define MEA_ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MEA_OK = 0,
+    MEA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, Nk == 0 with rows, non-finite scale */
+    MEA_ERR_UNSUPPORTED = 2,  /* head dim / dtype / direction outside the supported set */
+    MEA_ERR_MISALIGNED = 3,   /* a pointer violates the alignment rule above */
+    MEA_ERR_WORKSPACE = 4,    /* workspace missing or smaller than mea_attn_bwd_workspace_size */
+    MEA_ERR_CUDA = 5,         /* a CUDA runtime/driver call or a launch failed */
+    MEA_ERR_TIMEOUT = 6       /* a device-side bounded wait expired (see mea_last_device_error) */
+} mea_status_t;
+
+typedef enum {
+    MEA_DTYPE_F32 = 0,
+    MEA_DTYPE_BF16 = 1
+} mea_dtype_t;
+
+/*
+ * Forward pass: o = softmax(scale * q k^T) v and lse, per (batch, head).
+ *
+ * Source: "Self-attention Does Not Need O(n^2) Memory" (English summary),
+ * method bullets 1-4 (delayed normalisation, running maximum, key/value
+ * blocks summarised and merged); the two-block merge formulas of
+ * "当注意力成为瓶颈" (section IO感知).
+ *
+ * q,k,v   inputs (dtype), o output (dtype), lse output fp32 [B,H,Nq].
+ * B,H     batch and heads (>= 0); Nq query rows (>= 0); Nk keys (>= 1 when
+ *         B*H*Nq > 0); D head dim; scale multiplies q.k before the softmax.
+ * Nq == 0 or B == 0 or H == 0 is a no-op returning MEA_OK.
+ * Errors: MEA_ERR_INVALID_ARG, MEA_ERR_UNSUPPORTED, MEA_ERR_MISALIGNED,
+ *         MEA_ERR_CUDA (launch failure).
+ */
+mea_status_t mea_attn_fwd(const void* q, const void* k, const void* v,
+                          void* o, float* lse,
+                          int B, int H, int Nq, int Nk, int D, float scale,
+                          mea_dtype_t dtype, void* stream);
+
+/*
+ * Bytes of device workspace mea_attn_bwd needs for these sizes (written to
+ * *bytes): an fp32 dQ accumulator [B,H,Nq,D] and the fp32 row term
+ * D_i = sum_d dO_id O_id [B,H,Nq], each 256-byte aligned.  O(N*D), never
+ * O(N^2).  Errors: MEA_ERR_INVALID_ARG (null `bytes`, negative size),
+ * MEA_ERR_UNSUPPORTED (dtype/D not supported for backward).
+ */
+mea_status_t mea_attn_bwd_workspace_size(int B, int H, int Nq, int Nk, int D,
+                                         mea_dtype_t dtype, size_t* bytes);
+
+/*
+ * Backward pass: gradients of sum(dO o O) with respect to q, k, v.
+ *
+ * Source: "Self-attention Does Not Need O(n^2) Memory" (English summary),
+ * method bullet on differentiation: intermediate states are recomputed
+ * (checkpointing), here P = exp(scale * q k^T - lse) from the forward's lse.
+ * The gradient formulas are ordinary softmax calculus (the pages print none):
+ *   dV = P^T dO,  dP = dO V^T,  D_i = sum_d dO_id O_id,  dS = P o (dP - D),
+ *   dQ = scale dS K,  dK = scale dS^T Q.
+ *
+ * q,k,v,o,dO inputs (dtype); lse input fp32 [B,H,Nq] from mea_attn_fwd;
+ * dq,dk,dv outputs (dtype).  workspace: device memory of at least
+ * mea_attn_bwd_workspace_size() bytes, owned by the caller, contents on entry
+ * ignored, clobbered on exit.  dq is accumulated in fp32 with atomic adds, so it
+ * is not bitwise deterministic run to run (dk, dv are).
+ * Nq == 0 writes zeros to dk, dv.  Errors as for mea_attn_fwd plus
+ * MEA_ERR_WORKSPACE; MEA_DTYPE_F32 returns MEA_ERR_UNSUPPORTED.
+ */
+mea_status_t mea_attn_bwd(const void* q, const void* k, const void* v,
+                          const void* o, const float* lse, const void* dO,
+                          void* dq, void* dk, void* dv,
+                          int B, int H, int Nq, int Nk, int D, float scale,
+                          mea_dtype_t dtype,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's error
+ * flag.  Returns MEA_ERR_TIMEOUT if any kernel of this library gave up on a
+ * bounded wait since the last call, MEA_ERR_CUDA if the synchronisation
+ * itself failed, MEA_OK otherwise.
+ */
+mea_status_t mea_last_device_error(void* stream);
+
+/* Static, human-readable name of a status code (never NULL). */
+const char* mea_status_string(mea_status_t status);
+
+/*
+ * Text describing the most recent failure reported by this library on the
+ * calling host thread (which call failed and the CUDA error, if any); empty
+ * if none.  The pointer stays valid until the next call on the same thread.
+ */
+const char* mea_last_error_message(void);
+
+/* Library ABI version: 100 * major + minor. */
+int mea_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MEA_ATTN_H */

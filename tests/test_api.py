@@ -1,0 +1,130 @@
+"""Host-side tests of the C ABI (no kernel is launched).
+
+* the shared library builds, loads and exports every function that
+  include/mea_attn.h declares;
+* every invalid call is rejected with the documented status before any CUDA
+  call is made (fake device addresses are never dereferenced on the host);
+* the workspace size is O(N*D) and matches its documented layout.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mea_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from exact_memory_efficient_b200 import build as b
+    b.build()
+    import exact_memory_efficient_b200 as m
+    return m.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mea_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert {"mea_attn_fwd", "mea_attn_bwd", "mea_attn_bwd_workspace_size", "mea_last_device_error",
+            "mea_status_string", "mea_version"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in mea_attn.h but not exported"
+
+
+def test_status_strings(lib):
+    import exact_memory_efficient_b200 as m
+    for code in range(0, 7):
+        s = m.mea_status_string(code)
+        assert s.startswith("MEA_")
+    assert m.mea_status_string(99) == "MEA_ERR_UNKNOWN"
+    assert m.mea_version() == 100
+
+
+A = 0x10000  # fake, 16-byte aligned device addresses (never dereferenced on the host)
+BF16, F32 = 1, 0
+
+
+def fwd(lib, q=A, k=A, v=A, o=A, lse=A, B=1, H=1, Nq=16, Nk=16, D=64, scale=0.125, dtype=BF16):
+    return lib.mea_attn_fwd(q, k, v, o, lse, B, H, Nq, Nk, D, ctypes.c_float(scale), dtype, None)
+
+
+def bwd(lib, ptrs=None, B=1, H=1, Nq=16, Nk=16, D=64, scale=0.125, dtype=BF16, ws=A, ws_bytes=1 << 30):
+    p = [A] * 9 if ptrs is None else ptrs
+    return lib.mea_attn_bwd(*p, B, H, Nq, Nk, D, ctypes.c_float(scale), dtype, ws, ws_bytes, None)
+
+
+def test_forward_argument_validation(lib):
+    assert fwd(lib, q=None) == 1
+    assert fwd(lib, lse=None) == 1
+    assert fwd(lib, B=-1) == 1
+    assert fwd(lib, Nk=0) == 1
+    assert fwd(lib, D=0) == 1
+    assert fwd(lib, scale=float("nan")) == 1
+    assert fwd(lib, scale=float("inf")) == 1
+    assert fwd(lib, dtype=7) == 1
+    assert fwd(lib, D=96) == 2           # bf16 supports D in {64, 128}
+    assert fwd(lib, D=256) == 2
+    assert fwd(lib, D=48, dtype=F32) == 2  # fp32 needs D % 32 == 0 and D <= 128
+    assert fwd(lib, D=160, dtype=F32) == 2
+    assert fwd(lib, q=A + 8) == 3
+    assert fwd(lib, o=A + 4) == 3
+    assert fwd(lib, lse=A + 2) == 3
+
+
+def test_forward_empty_is_noop(lib):
+    # no rows: nothing is launched, so this succeeds without a GPU
+    assert fwd(lib, Nq=0) == 0
+    assert fwd(lib, B=0) == 0
+    assert fwd(lib, H=0, q=None) == 0
+
+
+def test_backward_argument_validation(lib):
+    assert bwd(lib, dtype=F32) == 2
+    assert bwd(lib, D=96) == 2
+    assert bwd(lib, Nk=0) == 1
+    assert bwd(lib, Nq=-3) == 1
+    ptrs = [A] * 9
+    ptrs[5] = None  # dO
+    assert bwd(lib, ptrs=ptrs) == 1
+    ptrs = [A] * 9
+    ptrs[7] = A + 8  # dk misaligned
+    assert bwd(lib, ptrs=ptrs) == 3
+    assert bwd(lib, ws=None) == 4
+    assert bwd(lib, ws_bytes=100) == 4
+    assert bwd(lib, ws=A + 16) == 3       # workspace must be 256-byte aligned
+    assert bwd(lib, B=0) == 0
+
+
+def test_workspace_size(lib):
+    out = ctypes.c_size_t(0)
+    assert lib.mea_attn_bwd_workspace_size(1, 16, 16384, 16384, 128, BF16, ctypes.byref(out)) == 0
+    rows = 16 * 16384
+    assert out.value == rows * 128 * 4 + rows * 4  # dQ accumulator + row term, both 256-aligned here
+    assert lib.mea_attn_bwd_workspace_size(2, 3, 5, 7, 64, BF16, ctypes.byref(out)) == 0
+    r = 2 * 3 * 5
+    assert out.value == ((r * 64 * 4 + 255) // 256) * 256 + ((r * 4 + 255) // 256) * 256
+    assert lib.mea_attn_bwd_workspace_size(1, 1, 4, 4, 64, F32, ctypes.byref(out)) == 2
+    assert lib.mea_attn_bwd_workspace_size(1, 1, 4, 4, 64, BF16, None) == 1
+    # O(N*D) extra memory, never O(N^2): doubling N doubles the workspace
+    a, b = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    lib.mea_attn_bwd_workspace_size(1, 1, 4096, 4096, 128, BF16, ctypes.byref(a))
+    lib.mea_attn_bwd_workspace_size(1, 1, 8192, 8192, 128, BF16, ctypes.byref(b))
+    assert b.value == 2 * a.value
+
+
+def test_python_binding_rejects_bad_tensors(lib):
+    import torch
+    import exact_memory_efficient_b200 as m
+    q = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16)
+    with pytest.raises(m.MeaError):
+        m.mea_attn_fwd(q, q, q, q, torch.zeros(1, 1, 4), 0.125)  # CPU tensors are rejected
+    with pytest.raises(m.MeaError):
+        m.mea_attn_fwd(q[0], q, q, q, torch.zeros(1, 1, 4), 0.125)

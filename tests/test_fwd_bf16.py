@@ -1,0 +1,133 @@
+"""bf16 tcgen05 forward against the fp64 oracle, through the C ABI (GPU).
+
+Full element-by-element comparison on shapes the oracle finishes in seconds
+(several 128-row tiles and ragged tails), and sampled rows at the full
+workload sizes, launched exactly as the bench launches them.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synthetic_inputs import custom, make_inputs, make_workload, to_f64
+from tests._parity import BF16_O, assert_close, assert_lse_close, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_fwd(q, k, v, scale):
+    import exact_memory_efficient_b200 as m
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    o, lse = m.attention_forward(qd, kd, vd, scale)
+    assert m.mea_last_device_error() == m.MEA_OK
+    return o, lse
+
+
+def full_check(q, k, v, scale, what, bf16_output=False):
+    o, lse = gpu_fwd(q, k, v, scale)
+    q64, k64, v64 = to_f64(q), to_f64(k), to_f64(v)
+    o_ref, lse_ref = oracle.attention_forward(q64, k64, v64, scale)
+    assert_close(to_np(o), o_ref, *BF16_O, what=f"O {what}", bf16_output=bf16_output)
+    assert_lse_close(to_np(lse), lse_ref, q64, k64, scale, what=f"lse {what}")
+
+
+@pytest.mark.parametrize("B,H,Nq,Nk,D", [
+    (1, 1, 128, 128, 64),
+    (1, 1, 256, 384, 128),
+    (2, 3, 300, 700, 64),     # ragged query and key tails, several tiles
+    (1, 2, 513, 257, 128),    # odd tile counts
+    (1, 1, 1, 1, 64),         # one row, one key
+    (1, 1, 1, 1000, 128),     # single query (decode-shaped)
+    (2, 2, 77, 5, 128),       # fewer keys than one tile
+    (1, 1, 1000, 1, 64),      # one key: O = V_0
+])
+def test_shapes_full(B, H, Nq, Nk, D):
+    w = custom(B, H, Nq, Nk, D, "bf16", backward=False)
+    q, k, v, _ = make_inputs(w, 11)
+    full_check(q, k, v, w.scale, f"{(B, H, Nq, Nk, D)}", bf16_output=True)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_encoder_512_full(seed):
+    w = make_workload("encoder_512_bf16")
+    q, k, v, _ = make_inputs(w, seed)
+    full_check(q, k, v, w.scale, f"encoder_512 seed {seed}")
+
+
+@pytest.mark.parametrize("name", ["mha_4k_bf16", "long_256_bf16", "long_1024_bf16", "long_4096_bf16",
+                                  "long_16384_bf16"])
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_workloads_sampled(name, seed):
+    """Full-size launch; oracle on sampled (batch, head, row) triples."""
+    w = make_workload(name)
+    q, k, v, _ = make_inputs(w, seed)
+    o, lse = gpu_fwd(q, k, v, w.scale)
+    o, lse = to_np(o), to_np(lse)
+    rng = np.random.default_rng(seed)
+    heads = {(0, 0), (w.B - 1, w.H - 1), (int(rng.integers(w.B)), int(rng.integers(w.H)))}
+    n_rows = min(w.Nq, 48)
+    for b, h in sorted(heads):
+        rows = np.unique(np.concatenate([[0, w.Nq - 1], rng.choice(w.Nq, n_rows, replace=False)]))
+        q64, k64, v64 = to_f64(q[b, h]), to_f64(k[b, h]), to_f64(v[b, h])
+        o_ref, lse_ref = oracle.attention_forward_rows(q64, k64, v64, w.scale, rows)
+        assert_close(o[b, h, rows], o_ref, *BF16_O, what=f"O {name} s{seed} ({b},{h})")
+        assert_lse_close(lse[b, h, rows], lse_ref, q64[rows], k64, w.scale, what=f"lse {name} ({b},{h})")
+
+
+def _grid(shape, gen, lo=-16, hi=16):
+    """Values on the 1/8 grid in [-2, 2]: exactly representable in bf16, also after adding small integers."""
+    return (torch.randint(lo, hi + 1, shape, generator=gen).float() / 8).to(torch.bfloat16)
+
+
+def test_shift_invariance():
+    """K -> K + 1 u^T: O unchanged, lse shifts by scale q.u (inputs exact in bf16)."""
+    g = torch.Generator().manual_seed(21)
+    Nq, Nk, D = 200, 300, 64
+    q, k = _grid((1, 2, Nq, D), g), _grid((1, 2, Nk, D), g)
+    v = torch.randn(1, 2, Nk, D, generator=g).to(torch.bfloat16)
+    u = torch.randint(-2, 3, (D,), generator=g).float()
+    k2 = (k.float() + u).to(torch.bfloat16)
+    assert torch.equal(k2.float(), k.float() + u)  # exact
+    o1, l1 = gpu_fwd(q, k, v, 0.125)
+    o2, l2 = gpu_fwd(q, k2, v, 0.125)
+    o1, o2, l1, l2 = to_np(o1), to_np(o2), to_np(l1), to_np(l2)
+    np.testing.assert_allclose(o2, o1, atol=2e-2)
+    shift = 0.125 * (to_f64(q) @ u.double().numpy())
+    np.testing.assert_allclose(l2 - l1, shift, atol=2e-3)
+
+
+def test_all_keys_equal():
+    g = torch.Generator().manual_seed(22)
+    Nq, Nk, D = 130, 1000, 128
+    q = torch.randn(1, 1, Nq, D, generator=g).to(torch.bfloat16)
+    k = torch.randn(1, 1, 1, D, generator=g).to(torch.bfloat16).expand(1, 1, Nk, D).contiguous()
+    v = torch.randn(1, 1, Nk, D, generator=g).to(torch.bfloat16)
+    o, lse = gpu_fwd(q, k, v, 1 / math.sqrt(D))
+    vbar = to_f64(v)[0, 0].mean(axis=0)
+    np.testing.assert_allclose(to_np(o)[0, 0], np.tile(vbar, (Nq, 1)), atol=2e-2)
+    expect = (to_f64(q)[0, 0] @ to_f64(k)[0, 0, 0]) / math.sqrt(D) + math.log(Nk)
+    np.testing.assert_allclose(to_np(lse)[0, 0], expect, atol=2e-3)
+
+
+def test_dominant_key_and_large_logits():
+    """One-hot keys scaled so one score beats the rest by > 50 (logits ~1e3)."""
+    D, Nk = 64, 64
+    a = 64.0
+    k = (torch.eye(D) * a).reshape(1, 1, Nk, D).to(torch.bfloat16)
+    perm = torch.tensor([5, 0, 63, 17, 17, 40] * 40)
+    q = (torch.eye(D)[perm] * 128.0).reshape(1, 1, -1, D).to(torch.bfloat16)  # score 64*128/8 = 1024
+    v = torch.randn(1, 1, Nk, D, generator=torch.Generator().manual_seed(23)).to(torch.bfloat16)
+    o, lse = gpu_fwd(q, k, v, 0.125)
+    np.testing.assert_allclose(to_np(o)[0, 0], to_f64(v)[0, 0][perm.numpy()], atol=1e-6)
+    np.testing.assert_allclose(to_np(lse)[0, 0], 1024.0, atol=1e-3)
+
+
+def test_deterministic():
+    w = custom(1, 4, 1000, 1000, 128, "bf16", backward=False)
+    q, k, v, _ = make_inputs(w, 3)
+    a, la = gpu_fwd(q, k, v, w.scale)
+    b, lb = gpu_fwd(q, k, v, w.scale)
+    assert torch.equal(a, b) and torch.equal(la, lb)
