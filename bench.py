@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Benchmark: exact attention forward + backward, bf16, n = 16384 (B1 H16 D128).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch: the bf16 forward
+(mea_attn_fwd) and the three backward phases (mea_attn_bwd_phase) on the
+long-sequence workload B=1, H=16, N=16384, D=128, synthetic N(0,1) inputs.
+The metric is TFLOP/s with the 4*B*H*N^2*D forward convention and 2.5x that
+for the backward; `value` is the whole-job throughput over all ranks (each
+rank runs its own independent batch: weak scaling, no data-path collective).
+
+Rank 0 prints one JSON line.  Under torchrun (N > 1) ranks synchronise with a
+barrier around the timed region and the slowest rank's device time is used.
+`--impl reference` times the fp64 CPU oracle (the only reference there is) on
+a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from synthetic_inputs import make_inputs, make_workload, custom  # noqa: E402
+
+WORKLOAD = "long_16384_bf16"
+METRIC = "attention fwd & fwd+bwd TFLOP/s, bf16 n=16384, % of B200 dense BF16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CSRC = os.path.join(ROOT, "exact_memory_efficient_b200", "csrc")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_sha() -> str:
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(CSRC, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current sources."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e or e.get("src_sha") != source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        power = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        loaded = [x for x in sm if x > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(power) if power else None}
+
+
+def cpu_oracle_sample(w, seed=0, q_rows=4096):
+    """Time the fp64 oracle's forward + backward on one head, q_rows query rows x all keys."""
+    import numpy as np
+    import oracle
+    from synthetic_inputs import to_f64
+    q, k, v, do = make_inputs(custom(1, 1, q_rows, w.Nk, w.D, "bf16", True, name="oracle_sample"), seed)
+    q2, k2, v2, do2 = (to_f64(x)[0, 0] for x in (q, k, v, do))
+    t0 = time.perf_counter()
+    oracle.attention_forward_2d(q2, k2, v2, w.scale)
+    oracle.attention_backward_2d(q2, k2, v2, do2, w.scale)
+    dt = time.perf_counter() - t0
+    flops = 3.5 * 4.0 * q_rows * w.Nk * w.D
+    cores = len(os.sched_getaffinity(0))
+    del np
+    return flops / dt / 1e12, dt, cores, (f"fp64 numpy oracle, forward then backward of 1 of {w.B * w.H} heads, "
+                                          f"{q_rows} of {w.Nq} query rows x all {w.Nk} keys, D={w.D}")
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = make_workload(WORKLOAD)
+    vals, times = [], []
+    cores, sample = None, None
+    for i in range(args.warmup + args.steps):
+        v, dt, cores, sample = cpu_oracle_sample(w, seed=i % 3)
+        if i >= args.warmup:
+            vals.append(v)
+            times.append(dt)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.median(times), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "N": w.Nq, "D": w.D, "sample": sample},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import exact_memory_efficient_b200 as m
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    m.load_library()
+    peaks, peak_src = load_peaks()
+    w = make_workload(args.workload)
+    if w.dtype != "bf16" or not w.backward:
+        raise SystemExit(f"--workload {args.workload}: the step needs a bf16 forward+backward workload")
+    scale = w.scale
+
+    # ---- inputs resident in HBM (one independent batch per rank)
+    q_h, k_h, v_h, do_h = make_inputs(w, seed=rank)
+    mem0 = torch.cuda.memory_allocated(dev)
+    q, k, v, do = (x.to(dev) for x in (q_h, k_h, v_h, do_h))
+    o = torch.empty_like(q)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    mem_io = torch.cuda.memory_allocated(dev) - mem0
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+    ws = torch.empty(m.mea_attn_bwd_workspace_size(w.B, w.H, w.Nq, w.Nk, w.D), dtype=torch.uint8, device=dev)
+    extra_bytes = lse.numel() * 4 + ws.numel()
+    stream = torch.cuda.current_stream()
+
+    def bwd(phase):
+        m.mea_attn_bwd_phase(phase, q, k, v, o, lse, do, dq, dk, dv, scale, ws, stream)
+
+    launches_per_step = 4  # fwd kernel + backward preprocess, main, finalise
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        m.mea_attn_fwd(q, k, v, o, lse, scale, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        bwd(m.MEA_BWD_PREPROCESS)
+        if ev is not None:
+            ev[2].record(stream)
+        bwd(m.MEA_BWD_MAIN)
+        if ev is not None:
+            ev[3].record(stream)
+        bwd(m.MEA_BWD_FINALIZE)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    st = m.mea_last_device_error(stream)
+    if st != m.MEA_OK:
+        raise RuntimeError(f"device error after warm-up: {m.mea_status_string(st)}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+    clocks.start()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    st = m.mea_last_device_error(stream)
+    if st != m.MEA_OK:
+        raise RuntimeError(f"device error in timed region: {m.mea_status_string(st)}")
+
+    total_ms = t_start.elapsed_time(t_end)
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    pre_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    main_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    fin_ms = [e[3].elapsed_time(e[4]) for e in evs]
+    t = torch.tensor([total_ms, sum(fwd_ms), sum(main_ms)], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, fwd_sum, main_sum = (float(x) for x in t.tolist())
+
+    fwd_flops = w.fwd_flops()
+    step_flops = 3.5 * fwd_flops
+    value = world * args.steps * step_flops / (total_ms * 1e-3) / 1e12
+    fwd_tf = fwd_flops / (statistics.mean(fwd_ms) * 1e-3) / 1e12
+    bwd_ms = [a + b + c for a, b, c in zip(pre_ms, main_ms, fin_ms)]
+    bwd_tf = 2.5 * fwd_flops / (statistics.mean(bwd_ms) * 1e-3) / 1e12
+    main_avg_ms = statistics.mean(main_ms)
+    main_tf = 2.5 * fwd_flops / (main_avg_ms * 1e-3) / 1e12
+
+    # The dominant kernel is the backward main kernel; it runs inside a step
+    # loop of total_ms; use the sustained GEMM peak once the loop is long.
+    sustained = total_ms >= 1000.0
+    peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    peak_step = peak
+
+    # ---- end to end through the public API with host buffers (pinned)
+    e2e = None
+    if not args.no_extras:
+        pin = [x.pin_memory() for x in (q_h, k_h, v_h, do_h)]
+        outs = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in (q_h, k_h, v_h, q_h)]
+        lse_h = torch.empty(lse.shape, dtype=torch.float32, pin_memory=True)
+        e2e_steps = max(1, min(args.steps, 5))
+
+        def e2e_step():
+            qd, kd, vd, dod = (x.to(dev, non_blocking=True) for x in pin)
+            od, lsed = m.attention_forward(qd, kd, vd, scale, stream)
+            dqd, dkd, dvd = m.attention_backward(qd, kd, vd, od, lsed, dod, scale, ws, stream)
+            for h, d_ in zip(outs, (od, dkd, dvd, dqd)):
+                h.copy_(d_, non_blocking=True)
+            lse_h.copy_(lsed, non_blocking=True)
+            torch.cuda.current_stream().synchronize()
+
+        e2e_step()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+        if dist is not None:
+            dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+        h2d = sum(x.numel() * x.element_size() for x in pin)
+        d2h = sum(x.numel() * x.element_size() for x in outs) + lse_h.numel() * 4
+        e2e = {"value": round(world * e2e_steps * step_flops / (float(e2e_ms.item()) * 1e-3) / 1e12, 3),
+               "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "steps": e2e_steps}
+
+    # ---- fp32 SIMT rows (secondary measurements, single-query HBM roofline)
+    rows = {}
+    if rank == 0:
+        rows[f"{w.name}_fwd"] = {"ms": round(statistics.mean(fwd_ms), 4), "TFLOP/s": round(fwd_tf, 1),
+                                 "frac_of_peak": round(fwd_tf / peak, 3)}
+        rows[f"{w.name}_bwd"] = {"ms": round(statistics.mean(bwd_ms), 4), "TFLOP/s": round(bwd_tf, 1),
+                                 "frac_of_peak": round(bwd_tf / peak, 3),
+                                 "phases_ms": {"preprocess": round(statistics.mean(pre_ms), 4),
+                                               "main": round(main_avg_ms, 4),
+                                               "finalize": round(statistics.mean(fin_ms), 4)}}
+    if rank == 0 and not args.no_extras:
+        ws1 = make_workload("single_query_f32")
+        q1, k1, v1, _ = (x.to(dev) if x is not None else None for x in make_inputs(ws1, 0))
+        o1, l1 = m.attention_forward(q1, k1, v1, ws1.scale)
+        for _ in range(5):
+            m.mea_attn_fwd(q1, k1, v1, o1, l1, ws1.scale)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 50
+        e0.record(stream)
+        for _ in range(reps):
+            m.mea_attn_fwd(q1, k1, v1, o1, l1, ws1.scale)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / reps
+        byts = (q1.numel() + k1.numel() + v1.numel() + o1.numel() + l1.numel()) * 4
+        rows["single_query_f32_fwd"] = {"us": round(us, 2), "GB/s": round(byts / (us * 1e-6) / 1e9, 1),
+                                        "frac_of_hbm": round(byts / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 3),
+                                        "note": "L2-warm back-to-back launches (67 MB working set < L2)"}
+        del q1, k1, v1, o1, l1
+
+    # ---- extra memory versus a materialised-scores attention (arithmetic)
+    naive_scores = w.B * w.H * w.Nq * w.Nk * 4
+    memory = {"extra_bytes_ours": extra_bytes, "io_bytes": mem_io,
+              "naive_score_matrix_fp32_bytes": naive_scores,
+              "naive_over_ours": round(naive_scores / extra_bytes, 1)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.no_extras:
+        cv, cdt, cores, sample = cpu_oracle_sample(w)
+        cpu = {"value": round(cv, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample,
+               "seconds": round(cdt, 2)}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.Nq, "D": w.D, "scale": scale,
+                       "global_batch": world * w.B, "seq_len": w.Nq, "parallelism": f"replicas x{world}",
+                       "step": "mea_attn_fwd + mea_attn_bwd (3 phases)",
+                       "l2": "inputs larger than L2 (q, k, v, o, dO, dq, dk, dv + fp32 dQ workspace), no flush"},
+            "pct_of_peak": round(100 * value / world / peak_step, 2),
+            "fwd_tflops": round(fwd_tf, 2), "bwd_tflops": round(bwd_tf, 2),
+            "roofline": {"kernel": f"bwd_main_kernel<{w.D}>", "bound": "tensor", "achieved": round(main_tf, 2),
+                         "peak": peak, "unit": "TFLOP/s", "frac": round(main_tf / peak, 4),
+                         "traffic": ncu_traffic(f"bwd_main_kernel<{w.D}>"),
+                         "peak_source": f"{peak_src} {'bf16_tflops_sustained' if sustained else 'bf16_tflops'}",
+                         "flops_per_launch": 2.5 * fwd_flops},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk, "memory": memory, "rows": rows, "src_sha": source_sha(),
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="workload name from synthetic_inputs.WORKLOADS (bf16 with backward); the default is the "
+                         "headline workload, others are for profiling captures")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the end-to-end, fp32-row and CPU-baseline measurements (profiling captures)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -23,7 +23,8 @@ __all__ = [
     "MeaError", "load_library", "library_path",
     "MEA_OK", "MEA_ERR_INVALID_ARG", "MEA_ERR_UNSUPPORTED", "MEA_ERR_MISALIGNED", "MEA_ERR_WORKSPACE",
     "MEA_ERR_CUDA", "MEA_ERR_TIMEOUT", "MEA_DTYPE_F32", "MEA_DTYPE_BF16",
-    "mea_attn_fwd", "mea_attn_bwd", "mea_attn_bwd_workspace_size", "mea_last_device_error",
+    "MEA_BWD_ALL", "MEA_BWD_PREPROCESS", "MEA_BWD_MAIN", "MEA_BWD_FINALIZE",
+    "mea_attn_fwd", "mea_attn_bwd", "mea_attn_bwd_phase", "mea_attn_bwd_workspace_size", "mea_last_device_error",
     "mea_status_string", "mea_last_error_message", "mea_version", "attention_forward", "attention_backward",
 ]
 
@@ -37,6 +38,11 @@ MEA_ERR_TIMEOUT = 6
 
 MEA_DTYPE_F32 = 0
 MEA_DTYPE_BF16 = 1
+
+MEA_BWD_ALL = 0
+MEA_BWD_PREPROCESS = 1
+MEA_BWD_MAIN = 2
+MEA_BWD_FINALIZE = 3
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -72,6 +78,8 @@ def load_library() -> ctypes.CDLL:
     lib.mea_attn_bwd_workspace_size.restype = i
     lib.mea_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
     lib.mea_attn_bwd.restype = i
+    lib.mea_attn_bwd_phase.argtypes = [i, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
+    lib.mea_attn_bwd_phase.restype = i
     lib.mea_last_device_error.argtypes = [vp]
     lib.mea_last_device_error.restype = i
     lib.mea_status_string.argtypes = [i]
@@ -154,6 +162,11 @@ def mea_attn_bwd_workspace_size(B: int, H: int, Nq: int, Nk: int, D: int, dtype=
 
 def mea_attn_bwd(q, k, v, o, lse, do, dq, dk, dv, scale: float, workspace, stream=None) -> None:
     """C ``mea_attn_bwd``: writes dq, dk, dv; ``workspace`` is a uint8 CUDA tensor."""
+    mea_attn_bwd_phase(MEA_BWD_ALL, q, k, v, o, lse, do, dq, dk, dv, scale, workspace, stream)
+
+
+def mea_attn_bwd_phase(phase: int, q, k, v, o, lse, do, dq, dk, dv, scale: float, workspace, stream=None) -> None:
+    """C ``mea_attn_bwd_phase``: one phase (MEA_BWD_*) of the backward pass."""
     B, H, Nq, D = _bhnd(q, "q")
     _, _, Nk, _ = _bhnd(k, "k")
     for name, t, shape in (("o", o, q.shape), ("do", do, q.shape), ("dq", dq, q.shape), ("v", v, k.shape),
@@ -161,10 +174,10 @@ def mea_attn_bwd(q, k, v, o, lse, do, dq, dk, dv, scale: float, workspace, strea
         if tuple(t.shape) != tuple(shape) or t.dtype != q.dtype:
             raise MeaError(MEA_ERR_INVALID_ARG, f"mea_attn_bwd: {name} shape/dtype mismatch")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = load_library().mea_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
-                                      _ptr(dv), B, H, Nq, Nk, D, float(scale), _dtype_code(q), _ptr(workspace),
-                                      ws_bytes, _stream_handle(stream))
-    _check(st, "mea_attn_bwd")
+    st = load_library().mea_attn_bwd_phase(int(phase), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do),
+                                            _ptr(dq), _ptr(dk), _ptr(dv), B, H, Nq, Nk, D, float(scale),
+                                            _dtype_code(q), _ptr(workspace), ws_bytes, _stream_handle(stream))
+    _check(st, "mea_attn_bwd_phase")
 
 
 def mea_last_device_error(stream=None) -> int:

@@ -203,9 +203,18 @@ mea_status_t mea_attn_bwd_workspace_size(int B, int H, int Nq, int Nk, int D, me
     return MEA_OK;
 }
 
-mea_status_t mea_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                          const void* dO, void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int D,
-                          float scale, mea_dtype_t dtype, void* workspace, size_t workspace_bytes, void* stream) {
+mea_status_t mea_attn_bwd_phase(mea_bwd_phase_t phase, const void* q, const void* k, const void* v, const void* o,
+                                const float* lse, const void* dO, void* dq, void* dk, void* dv, int B, int H, int Nq,
+                                int Nk, int D, float scale, mea_dtype_t dtype, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+    unsigned phases = 0;
+    switch (phase) {
+        case MEA_BWD_ALL: phases = mea::kBwdPhasePre | mea::kBwdPhaseMain | mea::kBwdPhaseFinal; break;
+        case MEA_BWD_PREPROCESS: phases = mea::kBwdPhasePre; break;
+        case MEA_BWD_MAIN: phases = mea::kBwdPhaseMain; break;
+        case MEA_BWD_FINALIZE: phases = mea::kBwdPhaseFinal; break;
+        default: return MEA_ERR_INVALID_ARG;
+    }
     mea_status_t st = common_checks(B, H, Nq, Nk, D, scale, dtype);
     if (st != MEA_OK) return st;
     if (dtype != MEA_DTYPE_BF16) return MEA_ERR_UNSUPPORTED;
@@ -213,7 +222,7 @@ mea_status_t mea_attn_bwd(const void* q, const void* k, const void* v, const voi
     if (BH == 0) return MEA_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (Nq == 0) {
-        if (Nk == 0) return MEA_OK;
+        if (Nk == 0 || !(phases & mea::kBwdPhaseMain)) return MEA_OK;
         if (!dk || !dv) return MEA_ERR_INVALID_ARG;
         if (!aligned16(dk) || !aligned16(dv)) return MEA_ERR_MISALIGNED;
         const size_t n = (size_t)BH * Nk * D * 2;
@@ -253,7 +262,14 @@ mea_status_t mea_attn_bwd(const void* q, const void* k, const void* v, const voi
     a.Nk = Nk;
     a.D = D;
     a.scale = scale;
-    return cuda_status(mea::launch_bwd_bf16(a, s), "bwd_bf16 launch");
+    return cuda_status(mea::launch_bwd_bf16(a, s, phases), "bwd_bf16 launch");
+}
+
+mea_status_t mea_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                          const void* dO, void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int D,
+                          float scale, mea_dtype_t dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    return mea_attn_bwd_phase(MEA_BWD_ALL, q, k, v, o, lse, dO, dq, dk, dv, B, H, Nq, Nk, D, scale, dtype,
+                              workspace, workspace_bytes, stream);
 }
 
 mea_status_t mea_last_device_error(void* stream) {

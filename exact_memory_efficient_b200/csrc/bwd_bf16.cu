@@ -423,19 +423,22 @@ cudaError_t launch_main(const Bf16BwdArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
-cudaError_t launch_bwd_bf16(const Bf16BwdArgs& a, cudaStream_t stream) {
+cudaError_t launch_bwd_bf16(const Bf16BwdArgs& a, cudaStream_t stream, unsigned phases) {
     const long long rows = (long long)a.BH * a.Nq;
-    if (rows > 0) {
+    if ((phases & kBwdPhasePre) && rows > 0) {
         const int warps = 8;
         const long long blocks = (rows + warps - 1) / warps;
         bwd_pre_kernel<<<(unsigned)blocks, 32 * warps, 0, stream>>>(a.o, a.dO, a.delta, a.dq_acc, rows, a.D);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    cudaError_t e = (a.D == 64) ? launch_main<64>(a, stream) : (a.D == 128) ? launch_main<128>(a, stream)
-                                                                              : cudaErrorInvalidValue;
-    if (e != cudaSuccess) return e;
-    if (rows > 0) {
+    cudaError_t e = cudaSuccess;
+    if (phases & kBwdPhaseMain) {
+        e = (a.D == 64) ? launch_main<64>(a, stream) : (a.D == 128) ? launch_main<128>(a, stream)
+                                                                    : cudaErrorInvalidValue;
+        if (e != cudaSuccess) return e;
+    }
+    if ((phases & kBwdPhaseFinal) && rows > 0) {
         const long long n4 = rows * a.D / 4;
         const int tpb = 256;
         bwd_dq_final_kernel<<<(unsigned)((n4 + tpb - 1) / tpb), tpb, 0, stream>>>(a.dq_acc, a.dq, n4, a.scale);

@@ -50,6 +50,10 @@ struct Bf16BwdArgs {
     int BH, Nq, Nk, D;
     float scale;
 };
-cudaError_t launch_bwd_bf16(const Bf16BwdArgs& a, cudaStream_t stream);
+// Phases of the backward, run in this order on one workspace.
+constexpr unsigned kBwdPhasePre = 1u;    // delta = rowsum(dO o O); dQ accumulator := 0
+constexpr unsigned kBwdPhaseMain = 2u;   // dK, dV; dQ accumulated in fp32
+constexpr unsigned kBwdPhaseFinal = 4u;  // dq = bf16(scale * dQ accumulator)
+cudaError_t launch_bwd_bf16(const Bf16BwdArgs& a, cudaStream_t stream, unsigned phases);
 
 }  // namespace mea

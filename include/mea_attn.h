@@ -122,6 +122,34 @@ mea_status_t mea_attn_bwd(const void* q, const void* k, const void* v,
                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The backward pass in its three stream-ordered phases, for callers that want
+ * to time or overlap them separately.  mea_attn_bwd(...) is exactly
+ * mea_attn_bwd_phase(MEA_BWD_ALL, ...).  Every phase takes the full argument
+ * list of mea_attn_bwd and validates it the same way; the phases must run in
+ * the order PREPROCESS, MAIN, FINALIZE on the same workspace:
+ *   MEA_BWD_PREPROCESS  D_i = sum_d dO_id O_id into the workspace; zeroes the
+ *                       fp32 dQ accumulator.               (reads o, dO)
+ *   MEA_BWD_MAIN        recomputes P from lse per key tile; writes dk, dv and
+ *                       adds dS K into the dQ accumulator.  (reads q, k, v, dO, lse)
+ *   MEA_BWD_FINALIZE    dq = bf16(scale * dQ accumulator). (writes dq)
+ * Errors as for mea_attn_bwd; an unknown phase returns MEA_ERR_INVALID_ARG.
+ */
+typedef enum {
+    MEA_BWD_ALL = 0,
+    MEA_BWD_PREPROCESS = 1,
+    MEA_BWD_MAIN = 2,
+    MEA_BWD_FINALIZE = 3
+} mea_bwd_phase_t;
+
+mea_status_t mea_attn_bwd_phase(mea_bwd_phase_t phase,
+                                const void* q, const void* k, const void* v,
+                                const void* o, const float* lse, const void* dO,
+                                void* dq, void* dk, void* dv,
+                                int B, int H, int Nq, int Nk, int D, float scale,
+                                mea_dtype_t dtype,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the current device's error
  * flag.  Returns MEA_ERR_TIMEOUT if any kernel of this library gave up on a
  * bounded wait since the last call, MEA_ERR_CUDA if the synchronisation

@@ -33,8 +33,8 @@ def declared_functions():
 
 def test_exports_every_declared_symbol(lib):
     names = declared_functions()
-    assert {"mea_attn_fwd", "mea_attn_bwd", "mea_attn_bwd_workspace_size", "mea_last_device_error",
-            "mea_status_string", "mea_version"} <= set(names)
+    assert {"mea_attn_fwd", "mea_attn_bwd", "mea_attn_bwd_phase", "mea_attn_bwd_workspace_size",
+            "mea_last_device_error", "mea_status_string", "mea_last_error_message", "mea_version"} <= set(names)
     for n in names:
         assert hasattr(lib, n), f"{n} declared in mea_attn.h but not exported"
 
@@ -101,6 +101,11 @@ def test_backward_argument_validation(lib):
     assert bwd(lib, ws_bytes=100) == 4
     assert bwd(lib, ws=A + 16) == 3       # workspace must be 256-byte aligned
     assert bwd(lib, B=0) == 0
+    # phased entry point: same validation, unknown phase rejected
+    assert lib.mea_attn_bwd_phase(9, *([A] * 9), 1, 1, 16, 16, 64, ctypes.c_float(0.125), BF16, A, 1 << 30,
+                                  None) == 1
+    assert lib.mea_attn_bwd_phase(2, *([A] * 9), 1, 1, 16, 16, 96, ctypes.c_float(0.125), BF16, A, 1 << 30,
+                                  None) == 2
 
 
 def test_workspace_size(lib):
