@@ -24,7 +24,7 @@ __all__ = [
     "MEA_OK", "MEA_ERR_INVALID_ARG", "MEA_ERR_UNSUPPORTED", "MEA_ERR_MISALIGNED", "MEA_ERR_WORKSPACE",
     "MEA_ERR_CUDA", "MEA_ERR_TIMEOUT", "MEA_DTYPE_F32", "MEA_DTYPE_BF16",
     "MEA_BWD_ALL", "MEA_BWD_PREPROCESS", "MEA_BWD_MAIN", "MEA_BWD_FINALIZE",
-    "mea_attn_fwd", "mea_attn_bwd", "mea_attn_bwd_phase", "mea_attn_bwd_workspace_size", "mea_last_device_error",
+    "mea_attn_fwd", "mea_attn_bwd", "mea_attn_bwd_phase", "mea_attn_bwd_workspace_size", "mea_attn_bwd_noalloc", "mea_last_device_error",
     "mea_status_string", "mea_last_error_message", "mea_version", "attention_forward", "attention_backward",
 ]
 
@@ -80,6 +80,8 @@ def load_library() -> ctypes.CDLL:
     lib.mea_attn_bwd.restype = i
     lib.mea_attn_bwd_phase.argtypes = [i, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
     lib.mea_attn_bwd_phase.restype = i
+    lib.mea_attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+    lib.mea_attn_bwd_noalloc.restype = i
     lib.mea_last_device_error.argtypes = [vp]
     lib.mea_last_device_error.restype = i
     lib.mea_status_string.argtypes = [i]
@@ -178,6 +180,21 @@ def mea_attn_bwd_phase(phase: int, q, k, v, o, lse, do, dq, dk, dv, scale: float
                                             _ptr(dq), _ptr(dk), _ptr(dv), B, H, Nq, Nk, D, float(scale),
                                             _dtype_code(q), _ptr(workspace), ws_bytes, _stream_handle(stream))
     _check(st, "mea_attn_bwd_phase")
+
+
+def mea_attn_bwd_noalloc(q, k, v, o, lse, do, dq, dk, dv, scale: float, stream=None) -> None:
+    """C ``mea_attn_bwd_noalloc``: the backward with the library's static scratch instead of a
+    caller workspace (for callers that cannot allocate; sizes up to a 64 MiB workspace)."""
+    B, H, Nq, D = _bhnd(q, "q")
+    _, _, Nk, _ = _bhnd(k, "k")
+    for name, t, shape in (("o", o, q.shape), ("do", do, q.shape), ("dq", dq, q.shape), ("v", v, k.shape),
+                           ("dk", dk, k.shape), ("dv", dv, k.shape)):
+        if tuple(t.shape) != tuple(shape) or t.dtype != q.dtype:
+            raise MeaError(MEA_ERR_INVALID_ARG, f"mea_attn_bwd_noalloc: {name} shape/dtype mismatch")
+    st = load_library().mea_attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq),
+                                              _ptr(dk), _ptr(dv), B, H, Nq, Nk, D, float(scale), _dtype_code(q),
+                                              _stream_handle(stream))
+    _check(st, "mea_attn_bwd_noalloc")
 
 
 def mea_last_device_error(stream=None) -> int:

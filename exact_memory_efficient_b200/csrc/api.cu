@@ -272,6 +272,60 @@ mea_status_t mea_attn_bwd(const void* q, const void* k, const void* v, const voi
                               workspace, workspace_bytes, stream);
 }
 
+// ---------------------------------------------------------------------------
+// Backward without any allocation, for callers that cannot allocate device
+// memory (see mea_attn_bwd_noalloc in mea_attn.h).  The scratch lives in one
+// file-scope device array that every device loading this library keeps until
+// the process exits; host code may only use its address as returned by
+// cudaGetSymbolAddress, never the array's name.
+}  // extern "C"
+
+namespace {
+constexpr size_t kNoAllocScratchBytes = (size_t)MEA_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+}  // namespace
+
+extern "C" {
+
+mea_status_t mea_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                  const void* dO, void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int D,
+                                  float scale, mea_dtype_t dtype, void* stream) {
+    mea_status_t st = common_checks(B, H, Nq, Nk, D, scale, dtype);
+    if (st != MEA_OK) return st;
+    if (dtype != MEA_DTYPE_BF16) return MEA_ERR_UNSUPPORTED;
+    size_t need = 0;
+    if ((st = mea_attn_bwd_workspace_size(B, H, Nq, Nk, D, dtype, &need)) != MEA_OK) return st;
+    if (need > kNoAllocScratchBytes) {
+        char buf[160];
+        std::snprintf(buf, sizeof(buf), "these sizes need %zu bytes of scratch; the static scratch holds %zu bytes",
+                      need, kNoAllocScratchBytes);
+        return fail(MEA_ERR_WORKSPACE, "mea_attn_bwd_noalloc", buf);
+    }
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail_cuda("cudaGetDevice", e);
+    if (dev < 0 || dev >= kMaxDevices) return MEA_ERR_UNSUPPORTED;
+    void* scratch = nullptr;
+    {
+        // One-time set-up per device, with that device current: resolve the
+        // device address of the static scratch array.
+        std::lock_guard<std::mutex> lk(g_noalloc_mu);
+        if (g_noalloc_ptr[dev] == nullptr) {
+            void* p = nullptr;
+            e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+            if (e != cudaSuccess || p == nullptr) return fail_cuda("cudaGetSymbolAddress(scratch)", e);
+            g_noalloc_ptr[dev] = p;
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    // The preprocess phase re-zeroes the dQ accumulator and rewrites the row
+    // term on every call, so nothing left by an earlier call is read.
+    return mea_attn_bwd_phase(MEA_BWD_ALL, q, k, v, o, lse, dO, dq, dk, dv, B, H, Nq, Nk, D, scale, dtype, scratch,
+                              kNoAllocScratchBytes, stream);
+}
+
 mea_status_t mea_last_device_error(void* stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail_cuda("cudaStreamSynchronize", e);

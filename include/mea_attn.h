@@ -150,6 +150,39 @@ mea_status_t mea_attn_bwd_phase(mea_bwd_phase_t phase,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Backward pass that allocates nothing and takes no workspace.  The paper has
+ * no counterpart: this is a deployment convenience of this library.
+ *
+ * Some callers cannot call cudaMalloc or any allocator: a plugin inside an
+ * inference runtime or framework whose device memory is owned and budgeted by
+ * the host application, real-time or embedded code whose memory is fixed at
+ * start-up, or code that holds no allocator handle at all.  For them the
+ * scratch that mea_attn_bwd takes as `workspace` (fp32 dQ accumulator and row
+ * term) lives in one static device array of MEA_NOALLOC_SCRATCH_BYTES (64 MiB)
+ * compiled into the library; every GPU that loads the library holds that array
+ * until the process exits.
+ *
+ * Arguments, layout, results and errors are those of mea_attn_bwd without the
+ * workspace pair.  Sizes whose workspace (mea_attn_bwd_workspace_size) exceeds
+ * MEA_NOALLOC_SCRATCH_BYTES are rejected with MEA_ERR_WORKSPACE and a message
+ * in mea_last_error_message().  The first call on each device resolves the
+ * array's device address (cudaGetSymbolAddress) with that device current; make
+ * that first call before any stream capture.  All calls on a device share the
+ * one array: calls that overlap on the GPU (different streams, or different
+ * host threads without ordering) race on it and give wrong gradients; calls
+ * ordered on one stream are safe.  Each call clears the part that must start
+ * at zero itself.  It never calls cudaMalloc, cudaFree or any allocating
+ * library routine.
+ */
+#define MEA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+mea_status_t mea_attn_bwd_noalloc(const void* q, const void* k, const void* v,
+                                  const void* o, const float* lse, const void* dO,
+                                  void* dq, void* dk, void* dv,
+                                  int B, int H, int Nq, int Nk, int D, float scale,
+                                  mea_dtype_t dtype, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the current device's error
  * flag.  Returns MEA_ERR_TIMEOUT if any kernel of this library gave up on a
  * bounded wait since the last call, MEA_ERR_CUDA if the synchronisation
