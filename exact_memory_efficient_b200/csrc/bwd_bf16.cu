@@ -16,7 +16,12 @@
 //                  dP^T = V dO_i^T         (smem x smem -> TMEM)
 //                  dV  += P^T dO_i         (P^T from TMEM, bf16)
 //                  dK  += dS^T Q_i         (dS^T from TMEM, bf16)
-//                  dQ_i = dS K             (dS from smem, bf16) -> fp32 atomic adds
+//                  dQ_i^T = K^T dS^T       (both from smem, bf16) -> fp32 atomic adds
+//                dQ is formed transposed so that TMEM lanes are head dims: the
+//                32 lanes of a warp then add to 32 consecutive floats of one dQ
+//                row (one 128-byte line per warp instruction).  For D = 64 the
+//                MMA still has M = 128; lanes 64..127 hold products with the V
+//                tile that follows K in shared memory and are ignored.
 //   bwd_dq_final dq = bf16(scale * dQacc).
 //
 // Roles in bwd_main (320 threads): warp 0 TMEM allocator and TMA producer (K, V
@@ -25,7 +30,7 @@
 // row 32*(w%4)+lane (the TMEM lane warp w can reach) and query half (w-2)/4 of
 // every tile.
 // TMEM: S^T [0,128)  dP^T [128,256)  dV [256,256+D)  dK [256+D, 256+2D)
-//       dQ: D=128 reuses the dP^T columns, D=64 uses [384,448).
+//       dQ^T (128 query columns): D=128 reuses the dP^T columns, D=64 uses [384,512).
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -96,7 +101,7 @@ struct BwdCfg {
     static constexpr int kSmemBytes = offBars + 256;
     static constexpr bool kDqInDp = (D == 128);
     static constexpr unsigned colS = 0, colDP = 128, colDV = 256, colDK = 256 + D;
-    static constexpr unsigned colDQ = kDqInDp ? 128u : 384u;
+    static constexpr unsigned colDQ = kDqInDp ? 128u : 384u;   // 128 columns (queries)
 };
 
 struct BwdBarriers {
@@ -122,9 +127,8 @@ __device__ __forceinline__ uint64_t mnmajor_desc(unsigned base, int kk) {
 // occupies columns [64 g, 64 g + 32) of its region.
 __device__ __forceinline__ unsigned packed_col(int kk) { return (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8; }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-                 : "memory");
+__device__ __forceinline__ void red_add_f32(float* addr, float a) {
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
 }
 
 template <int D>
@@ -217,20 +221,28 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (lane == 0) {
             constexpr unsigned idesc_t = make_idesc_bf16(128, 128, 0, 0);   // S^T, dP^T
             constexpr unsigned idesc_g = make_idesc_bf16(128, D, 0, 1);     // dV, dK (A in TMEM)
-            constexpr unsigned idesc_q = make_idesc_bf16(128, D, 1, 1);     // dQ (A = dS, MN-major)
+            constexpr unsigned idesc_q = make_idesc_bf16(128, 128, 1, 1);   // dQ^T (A = K^T, B = dS^T, MN-major)
             const unsigned aK = smem_u32(sK), aV = smem_u32(sV), aDS = smem_u32(sDS);
             bool ok = mbar_wait(&bars->kv_full, 0, abort_flag);
-            for (int i = 0; ok && i < n_q; ++i) {
-                const int st = i & 1;
-                if (!(ok = mbar_wait(&bars->q_full[st], (i >> 1) & 1, abort_flag))) break;
+            auto q_addr = [&](int i) -> unsigned { return smem_u32(sRing + (i & 1) * Cfg::kStageBytes); };
+            // S^T(i) = K Q_i^T into the S columns (once Q_i has landed)
+            auto issue_s = [&](int i) -> bool {
+                if (!mbar_wait(&bars->q_full[i & 1], (i >> 1) & 1, abort_flag)) return false;
                 tc_fence_after();
-                const unsigned aQ = smem_u32(sRing + st * Cfg::kStageBytes);
-                const unsigned aDO = aQ + Cfg::kKVBytes;
-                // S^T = K Q_i^T
+                const unsigned aQ = q_addr(i);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     mma_ss(tmem + Cfg::colS, kmajor_desc(aK, kk), kmajor_desc(aQ, kk), idesc_t, kk > 0);
                 mma_commit(&bars->s_full);
+                return true;
+            };
+            // Software pipeline: S^T(i+1) is issued right after dV(i) has been
+            // issued (which consumes P(i) from the same columns, in issue order),
+            // so the compute warps form P(i+1) while dK(i) and dQ(i) run.
+            if (ok) ok = issue_s(0);
+            for (int i = 0; ok && i < n_q; ++i) {
+                const unsigned aQ = q_addr(i);
+                const unsigned aDO = aQ + Cfg::kKVBytes;
                 // dP^T = V dO_i^T  (D=128: dP columns held dQ_{i-1} until the compute warps freed them)
                 if (Cfg::kDqInDp && i > 0) {
                     if (!(ok = mbar_wait(&bars->dq_free, (i - 1) & 1, abort_flag))) break;
@@ -247,7 +259,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int kk = 0; kk < kTile / 16; ++kk)
                     mma_ts(tmem + Cfg::colDV, tmem + Cfg::colS + packed_col(kk), mnmajor_desc(aDO, kk), idesc_g,
                            (i > 0 || kk > 0));
-                // dK += dS^T Q_i ; dQ_i = dS K
+                if (i + 1 < n_q && !(ok = issue_s(i + 1))) break;
+                // dK += dS^T Q_i ; dQ_i^T = K^T dS^T
                 if (!(ok = mbar_wait(&bars->ds_ready, i & 1, abort_flag))) break;
                 tc_fence_after();
 #pragma unroll
@@ -260,9 +273,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk)
-                    mma_ss(tmem + Cfg::colDQ, mnmajor_desc(aDS, kk), mnmajor_desc(aK, kk), idesc_q, kk > 0);
+                    mma_ss(tmem + Cfg::colDQ, mnmajor_desc(aK, kk), mnmajor_desc(aDS, kk), idesc_q, kk > 0);
                 mma_commit(&bars->dq_full);
-                mma_commit(&bars->q_empty[st]);
+                mma_commit(&bars->q_empty[i & 1]);
             }
             if (ok) mma_commit(&bars->final_done);
             mma_commit(&bars->drain);
@@ -287,60 +300,67 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         };
         float pre_l = 0.f, pre_d = 0.f;
         load_stats(0, pre_l, pre_d);
-        bool ok = true;
-        for (int i = 0; i < n_q; ++i) {
-            const int slot = i & 1;
+        float p[64];   // P^T of the current tile, fp32, kept for dS
+        // lse2 / delta of tile t into shared slot t&1 (all 256 compute threads)
+        auto stage_stats = [&](int t) -> bool {
+            const int slot = t & 1;
             if (ctid < 128) s_lse2[slot * kTile + ctid] = pre_l;
             else s_delta[slot * kTile + (ctid - 128)] = pre_d;
             mbar_arrive(&bars->stats[slot]);
-            if (!(ok = mbar_wait(&bars->stats[slot], (i >> 1) & 1, abort_flag))) break;
-            if (i + 1 < n_q) load_stats(i + 1, pre_l, pre_d);
-            const float* l2 = s_lse2 + slot * kTile + 64 * g;
-            const float* dl = s_delta + slot * kTile + 64 * g;
-
-            // ---- P^T = exp2(scale*log2e * S^T - lse2), query half g
-            if (!(ok = mbar_wait(&bars->s_full, i & 1, abort_flag))) break;
+            if (!mbar_wait(&bars->stats[slot], (t >> 1) & 1, abort_flag)) return false;
+            if (t + 1 < n_q) load_stats(t + 1, pre_l, pre_d);
+            return true;
+        };
+        // ---- P^T = exp2(scale*log2e * S^T - lse2), query half g
+        auto do_p = [&](int t) -> bool {
+            const float* l2 = s_lse2 + (t & 1) * kTile + 64 * g;
+            if (!mbar_wait(&bars->s_full, t & 1, abort_flag)) return false;
             tc_fence_after();
-            float p[64];
-            {
-                uint32_t sr[64];
-                tmem_ld32(tmem + lane_off + Cfg::colS + 64 * g, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                tmem_ld32(tmem + lane_off + Cfg::colS + 64 * g + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t sr[32];
+                tmem_ld32(tmem + lane_off + Cfg::colS + 64 * g + 32 * h, sr);
                 tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    p[c] = key_ok ? ex2_approx(fmaf(__uint_as_float(sr[c]), c_log2, -l2[c])) : 0.f;
-                uint32_t pk[32];
+                for (int c = 0; c < 32; ++c)
+                    p[32 * h + c] = key_ok ? ex2_approx(fmaf(__uint_as_float(sr[c]), c_log2, -l2[32 * h + c])) : 0.f;
+                uint32_t pk[16];
 #pragma unroll
-                for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
-                tmem_st32(tmem + lane_off + Cfg::colS + 64 * g, pk);
+                for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(p[32 * h + 2 * c], p[32 * h + 2 * c + 1]);
+                // packed P^T overwrites S^T columns this thread has already read
+                tmem_st16(tmem + lane_off + Cfg::colS + 64 * g + 16 * h, pk);
             }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars->p_ready);
-
-            // ---- dS^T = P^T o (dP^T - delta)
-            if (!(ok = mbar_wait(&bars->dp_full, i & 1, abort_flag))) break;
+            return true;
+        };
+        // ---- dS^T = P^T o (dP^T - delta): bf16 to TMEM (for dK) and to smem (for dQ)
+        auto do_ds = [&](int t) -> bool {
+            const float* dl = s_delta + (t & 1) * kTile + 64 * g;
+            if (!mbar_wait(&bars->dp_full, t & 1, abort_flag)) return false;
             tc_fence_after();
-            {
-                uint32_t dr[64];
-                tmem_ld32(tmem + lane_off + Cfg::colDP + 64 * g, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
-                tmem_ld32(tmem + lane_off + Cfg::colDP + 64 * g + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
-                tmem_wait_ld();
-                uint32_t pk[32];
+            // dS^T (keys x queries) in shared memory: MN-major operand, query block g,
+            // row = key, 16-byte chunk c of the 128-byte row swizzled by (key mod 8).
+            uint8_t* row = sDS + g * Cfg::kBoxBytes + kr * 128;
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const float d0 = p[2 * c] * (__uint_as_float(dr[2 * c]) - dl[2 * c]);
-                    const float d1 = p[2 * c + 1] * (__uint_as_float(dr[2 * c + 1]) - dl[2 * c + 1]);
+            for (int h = 0; h < 2; ++h) {
+                uint32_t dr[32];
+                tmem_ld32(tmem + lane_off + Cfg::colDP + 64 * g + 32 * h, dr);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const int q = 32 * h + 2 * c;
+                    const float d0 = p[q] * (__uint_as_float(dr[2 * c]) - dl[q]);
+                    const float d1 = p[q + 1] * (__uint_as_float(dr[2 * c + 1]) - dl[q + 1]);
                     pk[c] = pack_bf16x2(d0, d1);
                 }
-                tmem_st32(tmem + lane_off + Cfg::colDP + 64 * g, pk);
-                // dS (queries x keys) for the dQ MMA: MN-major A operand, query block g,
-                // row = key, 16-byte chunk c of the 128-byte row swizzled by (key mod 8).
-                uint8_t* row = sDS + g * Cfg::kBoxBytes + kr * 128;
+                // packed dS^T overwrites dP^T columns this thread has already read
+                tmem_st16(tmem + lane_off + Cfg::colDP + 64 * g + 16 * h, pk);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const int pc = c ^ (kr & 7);
+                for (int c = 0; c < 4; ++c) {
+                    const int pc = (4 * h + c) ^ (kr & 7);
                     *reinterpret_cast<uint4*>(row + pc * 16) =
                         make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
                 }
@@ -349,28 +369,37 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars->ds_ready);
-
-            // ---- dQacc[i] += dS K  (TMEM lanes are query rows here)
-            if (!(ok = mbar_wait(&bars->dq_full, i & 1, abort_flag))) break;
+            return true;
+        };
+        // ---- dQacc[t] += (K^T dS^T)^T: TMEM lane = head dim d, column = query
+        auto do_drain = [&](int t) -> bool {
+            if (!mbar_wait(&bars->dq_full, t & 1, abort_flag)) return false;
             tc_fence_after();
-            {
-                const int q_row = i * kTile + kr;
-                float* dst = dq_acc + ((size_t)bh * Nq + q_row) * D + g * (D / 2);
+            const int d = kr;                                   // this thread's lane
+            const int q0 = t * kTile + 64 * g;                  // first query of this half
+            float* dst = dq_acc + ((size_t)bh * Nq + q0) * D + d;
 #pragma unroll
-                for (int c0 = 0; c0 < D / 2; c0 += 32) {
-                    uint32_t qv[32];
-                    tmem_ld32(tmem + lane_off + Cfg::colDQ + g * (D / 2) + c0, qv);
-                    tmem_wait_ld();
-                    if (q_row < Nq) {
+            for (int c0 = 0; c0 < 64; c0 += 32) {
+                uint32_t qv[32];
+                tmem_ld32(tmem + lane_off + Cfg::colDQ + 64 * g + c0, qv);
+                tmem_wait_ld();
+                if (d < D) {
 #pragma unroll
-                        for (int c = 0; c < 32; c += 4)
-                            red_add_v4(dst + c0 + c, __uint_as_float(qv[c]), __uint_as_float(qv[c + 1]),
-                                       __uint_as_float(qv[c + 2]), __uint_as_float(qv[c + 3]));
-                    }
+                    for (int c = 0; c < 32; ++c)
+                        if (q0 + c0 + c < Nq) red_add_f32(dst + (size_t)(c0 + c) * D, __uint_as_float(qv[c]));
                 }
             }
             tc_fence_before();
             mbar_arrive(&bars->dq_free);
+            return true;
+        };
+        // Order per tile: dS(t), then P(t+1) (overlapping dK(t), dQ(t) on the
+        // tensor cores), then the dQ(t) drain.
+        bool ok = stage_stats(0) && do_p(0);
+        for (int i = 0; ok && i < n_q; ++i) {
+            if (!(ok = do_ds(i))) break;
+            if (i + 1 < n_q && !(ok = stage_stats(i + 1) && do_p(i + 1))) break;
+            if (!(ok = do_drain(i))) break;
         }
         // ---- epilogue: dV, dK (scaled) rows of this CTA's keys
         if (ok && mbar_wait(&bars->final_done, 0, abort_flag)) {
