@@ -25,7 +25,7 @@ __all__ = [
     "MEA_ERR_CUDA", "MEA_ERR_TIMEOUT", "MEA_DTYPE_F32", "MEA_DTYPE_BF16",
     "MEA_BWD_ALL", "MEA_BWD_PREPROCESS", "MEA_BWD_MAIN", "MEA_BWD_FINALIZE",
     "mea_attn_fwd", "mea_attn_bwd", "mea_attn_bwd_phase", "mea_attn_bwd_workspace_size", "mea_attn_bwd_noalloc", "mea_last_device_error",
-    "mea_status_string", "mea_last_error_message", "mea_version", "attention_forward", "attention_backward",
+    "mea_selftest_bounded_wait", "mea_status_string", "mea_last_error_message", "mea_version", "attention_forward", "attention_backward",
 ]
 
 MEA_OK = 0
@@ -82,6 +82,8 @@ def load_library() -> ctypes.CDLL:
     lib.mea_attn_bwd_phase.restype = i
     lib.mea_attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     lib.mea_attn_bwd_noalloc.restype = i
+    lib.mea_selftest_bounded_wait.argtypes = [vp, vp]
+    lib.mea_selftest_bounded_wait.restype = i
     lib.mea_last_device_error.argtypes = [vp]
     lib.mea_last_device_error.restype = i
     lib.mea_status_string.argtypes = [i]
@@ -195,6 +197,14 @@ def mea_attn_bwd_noalloc(q, k, v, o, lse, do, dq, dk, dv, scale: float, stream=N
                                               _ptr(dk), _ptr(dv), B, H, Nq, Nk, D, float(scale), _dtype_code(q),
                                               _stream_handle(stream))
     _check(st, "mea_attn_bwd_noalloc")
+
+
+def mea_selftest_bounded_wait(gave_up, stream=None) -> None:
+    """C ``mea_selftest_bounded_wait``: a kernel whose bounded wait must expire (about 1 s)."""
+    if gave_up.dtype != torch.int32 or not gave_up.is_cuda or gave_up.numel() < 1:
+        raise MeaError(MEA_ERR_INVALID_ARG, "gave_up must be an int32 CUDA tensor")
+    _check(load_library().mea_selftest_bounded_wait(_ptr(gave_up), _stream_handle(stream)),
+           "mea_selftest_bounded_wait")
 
 
 def mea_last_device_error(stream=None) -> int:

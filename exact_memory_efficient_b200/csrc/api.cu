@@ -12,10 +12,24 @@
 
 #include "kernels.h"
 #include "mea_attn.h"
+#include "ptx.cuh"
 
 namespace mea {
 __device__ unsigned int g_device_error = 0;
+
+// Self-test of the bounded wait: one thread waits on an mbarrier that nothing
+// will ever arrive on.  The wait gives up after its wall-clock limit, records
+// the timeout in g_device_error and the kernel returns normally.
+__global__ void selftest_wait_kernel(int* gave_up) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        const bool ok = mbar_wait(&bar, 0, nullptr);
+        *gave_up = ok ? 0 : 1;
+    }
 }
+}  // namespace mea
 
 namespace {
 
@@ -324,6 +338,16 @@ mea_status_t mea_attn_bwd_noalloc(const void* q, const void* k, const void* v, c
     // term on every call, so nothing left by an earlier call is read.
     return mea_attn_bwd_phase(MEA_BWD_ALL, q, k, v, o, lse, dO, dq, dk, dv, B, H, Nq, Nk, D, scale, dtype, scratch,
                               kNoAllocScratchBytes, stream);
+}
+
+mea_status_t mea_selftest_bounded_wait(int* gave_up, void* stream) {
+    if (gave_up == nullptr) return MEA_ERR_INVALID_ARG;
+    if (!aligned4(gave_up)) return MEA_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    mea_status_t st = device_info(&dev);
+    if (st != MEA_OK) return st;
+    mea::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(gave_up);
+    return cuda_status(cudaGetLastError(), "selftest launch");
 }
 
 mea_status_t mea_last_device_error(void* stream) {

@@ -190,6 +190,18 @@ mea_status_t mea_attn_bwd_noalloc(const void* q, const void* k, const void* v,
  */
 mea_status_t mea_last_device_error(void* stream);
 
+/*
+ * Self-test of the device-side failure detection.  Launches one kernel on
+ * `stream` whose only thread waits on an mbarrier that nothing ever completes,
+ * using the same bounded wait every kernel of this library uses.  After the
+ * wait's wall-clock limit (about one second) the kernel writes 1 to *gave_up
+ * (device memory, 4-byte aligned), records the expiry in the device error
+ * flag and returns normally: mea_last_device_error() then reports
+ * MEA_ERR_TIMEOUT and the context stays usable.  Nothing faults, traps or
+ * hangs.  Errors: MEA_ERR_INVALID_ARG, MEA_ERR_MISALIGNED, MEA_ERR_CUDA.
+ */
+mea_status_t mea_selftest_bounded_wait(int* gave_up, void* stream);
+
 /* Static, human-readable name of a status code (never NULL). */
 const char* mea_status_string(mea_status_t status);
 
