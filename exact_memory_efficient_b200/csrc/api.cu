@@ -111,6 +111,24 @@ mea_status_t make_map(CUtensorMap* m, const void* base, int BH, int N, int D) {
     return MEA_OK;
 }
 
+// 3-D fp32 map over the dQ accumulator [BH][Nq][D]: box {32, 64, 1}, no swizzle
+// (target of the backward's TMA reduce-adds; x offsets are multiples of 32 floats).
+mea_status_t make_map_f32_acc(CUtensorMap* m, void* base, int BH, int Nq, int D) {
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Nq, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)Nq * D * 4};
+    cuuint32_t box[3] = {32, 64, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        char buf[64];
+        std::snprintf(buf, sizeof(buf), "CUresult %d (dQ accumulator)", (int)r);
+        return fail(MEA_ERR_CUDA, "cuTensorMapEncodeTiled", buf);
+    }
+    return MEA_OK;
+}
+
 mea_status_t common_checks(int B, int H, int Nq, int Nk, int D, float scale, mea_dtype_t dtype) {
     if (dtype != MEA_DTYPE_F32 && dtype != MEA_DTYPE_BF16) return MEA_ERR_INVALID_ARG;
     if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || D <= 0) return MEA_ERR_INVALID_ARG;
@@ -270,6 +288,7 @@ mea_status_t mea_attn_bwd_phase(mea_bwd_phase_t phase, const void* q, const void
     a.dk = static_cast<uint16_t*>(dk);
     a.dv = static_cast<uint16_t*>(dv);
     a.dq_acc = static_cast<float*>(workspace);
+    if ((st = make_map_f32_acc(&a.tm_dq_acc, workspace, BH, Nq, D)) != MEA_OK) return st;
     a.delta = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round_up(rows * D * sizeof(float), 256));
     a.BH = BH;
     a.Nq = Nq;

@@ -16,19 +16,28 @@
 //                  dP^T = V dO_i^T         (smem x smem -> TMEM)
 //                  dV  += P^T dO_i         (P^T from TMEM, bf16)
 //                  dK  += dS^T Q_i         (dS^T from TMEM, bf16)
-//                  dQ_i^T = K^T dS^T       (both from smem, bf16) -> fp32 atomic adds
-//                dQ is formed transposed so that TMEM lanes are head dims: the
-//                32 lanes of a warp then add to 32 consecutive floats of one dQ
-//                row (one 128-byte line per warp instruction).  For D = 64 the
-//                MMA still has M = 128; lanes 64..127 hold products with the V
-//                tile that follows K in shared memory and are ignored.
+//                  dQ_i^T = K^T dS^T       (both from smem, bf16) -> fp32 TMA reduce-add
+//                dQ is formed transposed so that TMEM lanes are head dims: each
+//                warp of the dQ warpgroup stages [64 queries x 32 head dims] of
+//                it in shared memory and one TMA reduce-add sends it to the dQ
+//                accumulator.  For D = 64 the MMA still has M = 128; lanes
+//                64..127 hold products with the V tile that follows K in
+//                shared memory and are ignored.
 //   bwd_dq_final dq = bf16(scale * dQacc).
 //
-// Roles in bwd_main (320 threads): warp 0 TMEM allocator and TMA producer (K, V
-// once; Q_i, dO_i through a 2-stage ring; no multicast), warp 1 MMA issuer,
-// warps 2-9 two compute groups of four warps; thread (warp w, lane) owns key
-// row 32*(w%4)+lane (the TMEM lane warp w can reach) and query half (w-2)/4 of
-// every tile.
+// Roles in bwd_main (512 threads, four warpgroups):
+//   warp 0       TMEM allocator, then TMA producer (K, V once; Q_i, dO_i
+//                through a 2-stage ring; no multicast)
+//   warp 1       MMA issuer (one thread)
+//   warps 4-11   two compute warpgroups: thread (warp w, lane) owns key row
+//                32*(w%4)+lane (the TMEM lane warp w can reach) and query half
+//                (w-4)/4 of every tile: P^T and dS^T
+//   warps 12-15  dQ warpgroup: copies dQ_i^T out of TMEM (freeing it at once),
+//                stages it in shared memory and hands it to the TMA engine as
+//                fp32 reduce-adds into the dQ accumulator; also stages the
+//                lse / D values of later query tiles.
+// Every thread runs within 128 registers (512 threads x 128 = the register
+// file); P^T is kept in registers as packed bf16 pairs to make that fit.
 // TMEM: S^T [0,128)  dP^T [128,256)  dV [256,256+D)  dK [256+D, 256+2D)
 //       dQ^T (128 query columns): D=128 reuses the dP^T columns, D=64 uses [384,512).
 #include <cstdint>
@@ -42,8 +51,9 @@ namespace mea {
 namespace {
 
 constexpr int kTile = 128;
-constexpr int kThreads = 320;
+constexpr int kThreads = 512;
 constexpr int kComputeThreads = 256;
+constexpr int kDrainThreads = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------ pre
@@ -111,6 +121,7 @@ struct BwdBarriers {
     uint64_t s_full, dp_full, dq_full;
     uint64_t p_ready, ds_ready, dq_free;
     uint64_t stats[2];
+    uint64_t sds_free;
     uint64_t final_done;
     uint64_t drain;
     unsigned tmem_base;
@@ -127,17 +138,13 @@ __device__ __forceinline__ uint64_t mnmajor_desc(unsigned base, int kk) {
 // occupies columns [64 g, 64 g + 32) of its region.
 __device__ __forceinline__ unsigned packed_col(int kk) { return (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8; }
 
-__device__ __forceinline__ void red_add_f32(float* addr, float a) {
-    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
-}
-
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                const float* __restrict__ lse, const float* __restrict__ delta,
-                float* __restrict__ dq_acc, uint16_t* __restrict__ dk, uint16_t* __restrict__ dv,
-                int Nq, int Nk, float scale) {
+                const __grid_constant__ CUtensorMap tm_dq, const float* __restrict__ lse,
+                const float* __restrict__ delta, uint16_t* __restrict__ dk, uint16_t* __restrict__ dv, int Nq,
+                int Nk, float scale) {
     using Cfg = BwdCfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
     BwdBarriers* bars = reinterpret_cast<BwdBarriers*>(smem + Cfg::offBars);
@@ -165,9 +172,10 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(&bars->dq_full, 1);
         mbar_init(&bars->p_ready, kComputeThreads);
         mbar_init(&bars->ds_ready, kComputeThreads);
-        mbar_init(&bars->dq_free, kComputeThreads);
-        mbar_init(&bars->stats[0], kComputeThreads);
-        mbar_init(&bars->stats[1], kComputeThreads);
+        mbar_init(&bars->dq_free, kDrainThreads);
+        mbar_init(&bars->stats[0], kDrainThreads);
+        mbar_init(&bars->stats[1], kDrainThreads);
+        mbar_init(&bars->sds_free, 4);
         mbar_init(&bars->final_done, 1);
         mbar_init(&bars->drain, 1);
         bars->abort_flag = 0;
@@ -243,7 +251,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int i = 0; ok && i < n_q; ++i) {
                 const unsigned aQ = q_addr(i);
                 const unsigned aDO = aQ + Cfg::kKVBytes;
-                // dP^T = V dO_i^T  (D=128: dP columns held dQ_{i-1} until the compute warps freed them)
+                // dP^T = V dO_i^T  (D=128: dP columns held dQ_{i-1} until the dQ warps copied it out)
                 if (Cfg::kDqInDp && i > 0) {
                     if (!(ok = mbar_wait(&bars->dq_free, (i - 1) & 1, abort_flag))) break;
                     tc_fence_after();
@@ -281,39 +289,19 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mma_commit(&bars->drain);
             mbar_wait(&bars->drain, 0, nullptr);
         }
-    } else {
+    } else if (warp >= 4 && warp < 12) {
         // ------------------------------------------------ compute warps
-        const int g = (warp - 2) >> 2;                 // query half of every tile
+        const int g = (warp - 4) >> 2;                 // query half of every tile
         const unsigned sub = warp & 3;
         const int kr = sub * 32 + lane;                // key row within the tile (TMEM lane)
         const unsigned lane_off = (sub * 32u) << 16;
-        const int ctid = threadIdx.x - 64;             // 0..255
         const float c_log2 = scale * kLog2e;
         const bool key_ok = (n0 + kr) < Nk;
-        const float* lse_h = lse + (size_t)bh * Nq;
-        const float* delta_h = delta + (size_t)bh * Nq;
-        // stage lse2 / delta of tile 0
-        auto load_stats = [&](int i, float& lv, float& dvv) {
-            const int row = i * kTile + (ctid & 127);
-            lv = (row < Nq) ? lse_h[row] * kLog2e : INFINITY;
-            dvv = (row < Nq) ? delta_h[row] : 0.f;
-        };
-        float pre_l = 0.f, pre_d = 0.f;
-        load_stats(0, pre_l, pre_d);
-        float p[64];   // P^T of the current tile, fp32, kept for dS
-        // lse2 / delta of tile t into shared slot t&1 (all 256 compute threads)
-        auto stage_stats = [&](int t) -> bool {
-            const int slot = t & 1;
-            if (ctid < 128) s_lse2[slot * kTile + ctid] = pre_l;
-            else s_delta[slot * kTile + (ctid - 128)] = pre_d;
-            mbar_arrive(&bars->stats[slot]);
-            if (!mbar_wait(&bars->stats[slot], (t >> 1) & 1, abort_flag)) return false;
-            if (t + 1 < n_q) load_stats(t + 1, pre_l, pre_d);
-            return true;
-        };
+        uint32_t pp[32];   // P^T of the current tile as packed bf16 pairs (exactly what dV used)
         // ---- P^T = exp2(scale*log2e * S^T - lse2), query half g
         auto do_p = [&](int t) -> bool {
             const float* l2 = s_lse2 + (t & 1) * kTile + 64 * g;
+            if (!mbar_wait(&bars->stats[t & 1], (t >> 1) & 1, abort_flag)) return false;
             if (!mbar_wait(&bars->s_full, t & 1, abort_flag)) return false;
             tc_fence_after();
 #pragma unroll
@@ -322,13 +310,14 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tmem_ld32(tmem + lane_off + Cfg::colS + 64 * g + 32 * h, sr);
                 tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 32; ++c)
-                    p[32 * h + c] = key_ok ? ex2_approx(fmaf(__uint_as_float(sr[c]), c_log2, -l2[32 * h + c])) : 0.f;
-                uint32_t pk[16];
-#pragma unroll
-                for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(p[32 * h + 2 * c], p[32 * h + 2 * c + 1]);
+                for (int c = 0; c < 16; ++c) {
+                    const float p0 = key_ok ? ex2_approx(fmaf(__uint_as_float(sr[2 * c]), c_log2, -l2[32 * h + 2 * c])) : 0.f;
+                    const float p1 =
+                        key_ok ? ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), c_log2, -l2[32 * h + 2 * c + 1])) : 0.f;
+                    pp[16 * h + c] = pack_bf16x2(p0, p1);
+                }
                 // packed P^T overwrites S^T columns this thread has already read
-                tmem_st16(tmem + lane_off + Cfg::colS + 64 * g + 16 * h, pk);
+                tmem_st16(tmem + lane_off + Cfg::colS + 64 * g + 16 * h, *reinterpret_cast<const uint32_t(*)[16]>(&pp[16 * h]));
             }
             tmem_wait_st();
             tc_fence_before();
@@ -339,6 +328,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         auto do_ds = [&](int t) -> bool {
             const float* dl = s_delta + (t & 1) * kTile + 64 * g;
             if (!mbar_wait(&bars->dp_full, t & 1, abort_flag)) return false;
+            // the dQ warps staged dQ_{t-1} in the dS buffer until this phase
+            if (t > 0 && !mbar_wait(&bars->sds_free, (t - 1) & 1, abort_flag)) return false;
             tc_fence_after();
             // dS^T (keys x queries) in shared memory: MN-major operand, query block g,
             // row = key, 16-byte chunk c of the 128-byte row swizzled by (key mod 8).
@@ -352,8 +343,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
                     const int q = 32 * h + 2 * c;
-                    const float d0 = p[q] * (__uint_as_float(dr[2 * c]) - dl[q]);
-                    const float d1 = p[q + 1] * (__uint_as_float(dr[2 * c + 1]) - dl[q + 1]);
+                    const uint32_t pr = pp[16 * h + c];
+                    const float d0 = __uint_as_float(pr << 16) * (__uint_as_float(dr[2 * c]) - dl[q]);
+                    const float d1 = __uint_as_float(pr & 0xffff0000u) * (__uint_as_float(dr[2 * c + 1]) - dl[q + 1]);
                     pk[c] = pack_bf16x2(d0, d1);
                 }
                 // packed dS^T overwrites dP^T columns this thread has already read
@@ -371,35 +363,12 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_arrive(&bars->ds_ready);
             return true;
         };
-        // ---- dQacc[t] += (K^T dS^T)^T: TMEM lane = head dim d, column = query
-        auto do_drain = [&](int t) -> bool {
-            if (!mbar_wait(&bars->dq_full, t & 1, abort_flag)) return false;
-            tc_fence_after();
-            const int d = kr;                                   // this thread's lane
-            const int q0 = t * kTile + 64 * g;                  // first query of this half
-            float* dst = dq_acc + ((size_t)bh * Nq + q0) * D + d;
-#pragma unroll
-            for (int c0 = 0; c0 < 64; c0 += 32) {
-                uint32_t qv[32];
-                tmem_ld32(tmem + lane_off + Cfg::colDQ + 64 * g + c0, qv);
-                tmem_wait_ld();
-                if (d < D) {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        if (q0 + c0 + c < Nq) red_add_f32(dst + (size_t)(c0 + c) * D, __uint_as_float(qv[c]));
-                }
-            }
-            tc_fence_before();
-            mbar_arrive(&bars->dq_free);
-            return true;
-        };
         // Order per tile: dS(t), then P(t+1) (overlapping dK(t), dQ(t) on the
-        // tensor cores), then the dQ(t) drain.
-        bool ok = stage_stats(0) && do_p(0);
+        // tensor cores); the dQ warps drain dQ(t) meanwhile.
+        bool ok = do_p(0);
         for (int i = 0; ok && i < n_q; ++i) {
             if (!(ok = do_ds(i))) break;
-            if (i + 1 < n_q && !(ok = stage_stats(i + 1) && do_p(i + 1))) break;
-            if (!(ok = do_drain(i))) break;
+            if (i + 1 < n_q && !(ok = do_p(i + 1))) break;
         }
         // ---- epilogue: dV, dK (scaled) rows of this CTA's keys
         if (ok && mbar_wait(&bars->final_done, 0, abort_flag)) {
@@ -427,6 +396,64 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             }
         }
+    } else if (warp >= 12) {
+        // ------------------------------------------------ dQ warps (+ lse/D staging)
+        const unsigned sub = warp & 3;
+        const int d = sub * 32 + lane;                 // TMEM lane = head dim of dQ^T
+        const unsigned lane_off = (sub * 32u) << 16;
+        const bool active = d < D;                     // D = 64: lanes 64..127 hold nothing useful
+        const int j = threadIdx.x - 384;               // 0..127
+        const float* lse_h = lse + (size_t)bh * Nq;
+        const float* delta_h = delta + (size_t)bh * Nq;
+        float* stage = reinterpret_cast<float*>(sDS + sub * 8192);   // this warp: 64 rows x 32 floats
+        auto stage_stats = [&](int t) {
+            const int row = t * kTile + j;
+            s_lse2[(t & 1) * kTile + j] = (row < Nq) ? lse_h[row] * kLog2e : INFINITY;
+            s_delta[(t & 1) * kTile + j] = (row < Nq) ? delta_h[row] : 0.f;
+            mbar_arrive(&bars->stats[t & 1]);
+        };
+        // one half (64 queries) of dQ^T from registers to this warp's staging
+        // buffer as [query][32 head dims], then one TMA reduce-add (not waited for)
+        auto stage_and_reduce = [&](const uint32_t (&v)[64], int q0) {
+            if (active) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) stage[c * 32 + lane] = __uint_as_float(v[c]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && active && q0 < Nq) {
+                tma_reduce_add_3d(&tm_dq, stage, 32 * sub, q0, bh);
+                bulk_commit_group();
+            }
+        };
+        auto staging_reusable = [&]() {                // the TMA engine has read the staging buffer
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+        };
+        stage_stats(0);
+        if (n_q > 1) stage_stats(1);
+        bool ok = true;
+        for (int t = 0; ok && t < n_q; ++t) {
+            if (!(ok = mbar_wait(&bars->dq_full, t & 1, abort_flag))) break;
+            tc_fence_after();
+            uint32_t v[64];
+            tmem_ld32(tmem + lane_off + Cfg::colDQ, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+            tmem_ld32(tmem + lane_off + Cfg::colDQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+            tmem_wait_ld();
+            stage_and_reduce(v, t * kTile);
+            tmem_ld32(tmem + lane_off + Cfg::colDQ + 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+            tmem_ld32(tmem + lane_off + Cfg::colDQ + 96, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&bars->dq_free);               // dQ^T columns may be overwritten now
+            // tile t's lse/D are no longer read (dS(t) is done): slot t&1 takes tile t+2
+            if (t + 2 < n_q) stage_stats(t + 2);
+            staging_reusable();
+            stage_and_reduce(v, t * kTile + 64);
+            staging_reusable();
+            if (lane == 0) mbar_arrive(&bars->sds_free);   // the dS buffer is free for dS(t+1)
+        }
+        if (lane == 0) bulk_wait_all();                // every reduce-add has completed
     }
 
     tc_fence_before();
@@ -445,7 +472,7 @@ cudaError_t launch_main(const Bf16BwdArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
     dim3 grid((a.Nk + kTile - 1) / kTile, a.BH, 1);
-    kern<<<grid, kThreads, Cfg::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.lse, a.delta, a.dq_acc,
+    kern<<<grid, kThreads, Cfg::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.tm_dq_acc, a.lse, a.delta,
                                                       a.dk, a.dv, a.Nq, a.Nk, a.scale);
     return cudaGetLastError();
 }

@@ -39,6 +39,7 @@ cudaError_t launch_fwd_bf16(const Bf16FwdArgs& a, cudaStream_t stream);
 // bf16 backward (bwd_bf16.cu).
 struct Bf16BwdArgs {
     CUtensorMap tm_q, tm_k, tm_v, tm_do;
+    CUtensorMap tm_dq_acc;  // fp32 {D, Nq, BH}, box {32, 64, 1}, no swizzle (TMA reduce-add target)
     const uint16_t* o;
     const uint16_t* dO;
     const float* lse;
