@@ -26,16 +26,18 @@
 //   bwd_dq_final dq = bf16(scale * dQacc).
 //
 // Roles in bwd_main (512 threads, four warpgroups):
-//   warp 0       TMEM allocator, then TMA producer (K, V once; Q_i, dO_i
-//                through a 2-stage ring; no multicast)
+//   warp 0       TMEM allocator, then TMA producer (K, V once; then Q_i, dO_i;
+//                no multicast)
 //   warp 1       MMA issuer (one thread)
 //   warps 4-11   two compute warpgroups: thread (warp w, lane) owns key row
 //                32*(w%4)+lane (the TMEM lane warp w can reach) and query half
 //                (w-4)/4 of every tile: P^T and dS^T
 //   warps 12-15  dQ warpgroup: copies dQ_i^T out of TMEM (freeing it at once),
-//                stages it in shared memory and hands it to the TMA engine as
-//                fp32 reduce-adds into the dQ accumulator; also stages the
-//                lse / D values of later query tiles.
+//                stages it in its own shared-memory buffer and hands it to the
+//                TMA engine as fp32 reduce-adds into the dQ accumulator; also
+//                stages the lse / D values of later query tiles.
+// Shared memory (D = 128): K, V 32 KB each; Q ring 2 x 32 KB; dO 32 KB (one
+// buffer: dead after dV(i)); dS^T 32 KB; dQ staging 32 KB; lse/D 2 KB.
 // Every thread runs within 128 registers (512 threads x 128 = the register
 // file); P^T is kept in registers as packed bf16 pairs to make that fit.
 // TMEM: S^T [0,128)  dP^T [128,256)  dV [256,256+D)  dK [256+D, 256+2D)
@@ -98,15 +100,16 @@ __global__ void bwd_dq_final_kernel(const float* __restrict__ dq_acc, uint16_t* 
 template <int D>
 struct BwdCfg {
     static constexpr int kKVBytes = kTile * D * 2;      // one K (or V, Q, dO) tile
-    static constexpr int kStageBytes = 2 * kKVBytes;    // Q_i + dO_i
-    static constexpr int kStages = 2;
-    static constexpr int kDSBytes = kTile * kTile * 2;  // dS tile, bf16
+    static constexpr int kDSBytes = kTile * kTile * 2;  // dS^T tile, bf16
+    static constexpr int kStageBytes = 4 * 64 * 32 * 4; // dQ staging: 4 warps x [64 queries x 32 floats]
     static constexpr int kBoxBytes = 128 * 128;
     static constexpr int offK = 0;
-    static constexpr int offV = kKVBytes;
-    static constexpr int offRing = 2 * kKVBytes;
-    static constexpr int offDS = offRing + kStages * kStageBytes;
-    static constexpr int offStats = offDS + kDSBytes;          // lse2[2][128], delta[2][128]
+    static constexpr int offV = kKVBytes;               // must follow K (read as K^T rows 64..127 at D = 64)
+    static constexpr int offQ = 2 * kKVBytes;           // Q_i ring, 2 stages
+    static constexpr int offDO = offQ + 2 * kKVBytes;   // dO_i, single buffer (dead after dV(i))
+    static constexpr int offDS = offDO + kKVBytes;
+    static constexpr int offStage = offDS + kDSBytes;
+    static constexpr int offStats = offStage + kStageBytes;    // lse2[2][128], delta[2][128]
     static constexpr int offBars = offStats + 4 * kTile * 4;
     static constexpr int kSmemBytes = offBars + 256;
     static constexpr bool kDqInDp = (D == 128);
@@ -118,10 +121,10 @@ struct BwdBarriers {
     uint64_t kv_full;
     uint64_t q_full[2];
     uint64_t q_empty[2];
+    uint64_t do_full, do_empty;
     uint64_t s_full, dp_full, dq_full;
     uint64_t p_ready, ds_ready, dq_free;
     uint64_t stats[2];
-    uint64_t sds_free;
     uint64_t final_done;
     uint64_t drain;
     unsigned tmem_base;
@@ -167,6 +170,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&bars->q_full[s], 1);
             mbar_init(&bars->q_empty[s], 1);
         }
+        mbar_init(&bars->do_full, 1);
+        mbar_init(&bars->do_empty, 1);
         mbar_init(&bars->s_full, 1);
         mbar_init(&bars->dp_full, 1);
         mbar_init(&bars->dq_full, 1);
@@ -175,7 +180,6 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(&bars->dq_free, kDrainThreads);
         mbar_init(&bars->stats[0], kDrainThreads);
         mbar_init(&bars->stats[1], kDrainThreads);
-        mbar_init(&bars->sds_free, 4);
         mbar_init(&bars->final_done, 1);
         mbar_init(&bars->drain, 1);
         bars->abort_flag = 0;
@@ -192,8 +196,10 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     volatile int* abort_flag = &bars->abort_flag;
     uint8_t* sK = smem + Cfg::offK;
     uint8_t* sV = smem + Cfg::offV;
-    uint8_t* sRing = smem + Cfg::offRing;
+    uint8_t* sQ = smem + Cfg::offQ;
+    uint8_t* sDO = smem + Cfg::offDO;
     uint8_t* sDS = smem + Cfg::offDS;
+    uint8_t* sStage = smem + Cfg::offStage;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -207,21 +213,41 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tma_load_3d(sK + b * Cfg::kBoxBytes, &tm_k, &bars->kv_full, b * 64, n0, bh);
                 tma_load_3d(sV + b * Cfg::kBoxBytes, &tm_v, &bars->kv_full, b * 64, n0, bh);
             }
-            int issued = 0;
+            // Q_i: 2-stage ring (Q_{i+1} is read by S^T(i+1) before dK(i) frees Q_i).
+            // dO_i: single buffer, reloaded once dV(i) and dP^T(i) have read it.
+            auto load_q = [&](int i) {
+                mbar_arrive_expect_tx(&bars->q_full[i & 1], Cfg::kKVBytes);
+                for (int b = 0; b < D / 64; ++b)
+                    tma_load_3d(sQ + (i & 1) * Cfg::kKVBytes + b * Cfg::kBoxBytes, &tm_q, &bars->q_full[i & 1],
+                                b * 64, i * kTile, bh);
+            };
+            auto load_do = [&](int i) {
+                mbar_arrive_expect_tx(&bars->do_full, Cfg::kKVBytes);
+                for (int b = 0; b < D / 64; ++b)
+                    tma_load_3d(sDO + b * Cfg::kBoxBytes, &tm_do, &bars->do_full, b * 64, i * kTile, bh);
+            };
+            // dO_{i+1} is issued as soon as dV(i) has read dO_i, before Q_{i+2}
+            // (whose buffer frees only after dQ(i)).
+            int q_issued = 1, do_issued = 1;
+            load_q(0);
+            load_do(0);
+            if (n_q > 1) { load_q(1); q_issued = 2; }
             for (int i = 0; i < n_q; ++i) {
-                const int st = i & 1;
-                if (i >= 2 && !mbar_wait(&bars->q_empty[st], ((i >> 1) - 1) & 1, abort_flag)) break;
-                uint8_t* dst = sRing + st * Cfg::kStageBytes;
-                mbar_arrive_expect_tx(&bars->q_full[st], Cfg::kStageBytes);
-                for (int b = 0; b < D / 64; ++b) {
-                    tma_load_3d(dst + b * Cfg::kBoxBytes, &tm_q, &bars->q_full[st], b * 64, i * kTile, bh);
-                    tma_load_3d(dst + Cfg::kKVBytes + b * Cfg::kBoxBytes, &tm_do, &bars->q_full[st], b * 64,
-                                i * kTile, bh);
+                if (i + 1 < n_q) {
+                    if (!mbar_wait(&bars->do_empty, i & 1, abort_flag)) break;
+                    load_do(i + 1);
+                    do_issued = i + 2;
                 }
-                issued = i + 1;
+                if (i + 2 < n_q) {
+                    if (!mbar_wait(&bars->q_empty[i & 1], (i >> 1) & 1, abort_flag)) break;
+                    load_q(i + 2);
+                    q_issued = i + 3;
+                }
             }
-            for (int i = (issued > 2 ? issued - 2 : 0); i < issued; ++i)
+            // Never leave with copies in flight: wait until the last loads landed.
+            for (int i = (q_issued > 2 ? q_issued - 2 : 0); i < q_issued; ++i)
                 mbar_wait(&bars->q_full[i & 1], (i >> 1) & 1, nullptr);
+            if (do_issued > 0) mbar_wait(&bars->do_full, (do_issued - 1) & 1, nullptr);
             mbar_wait(&bars->kv_full, 0, nullptr);
         }
     } else if (warp == 1) {
@@ -232,7 +258,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             constexpr unsigned idesc_q = make_idesc_bf16(128, 128, 1, 1);   // dQ^T (A = K^T, B = dS^T, MN-major)
             const unsigned aK = smem_u32(sK), aV = smem_u32(sV), aDS = smem_u32(sDS);
             bool ok = mbar_wait(&bars->kv_full, 0, abort_flag);
-            auto q_addr = [&](int i) -> unsigned { return smem_u32(sRing + (i & 1) * Cfg::kStageBytes); };
+            auto q_addr = [&](int i) -> unsigned { return smem_u32(sQ + (i & 1) * Cfg::kKVBytes); };
+            const unsigned aDO = smem_u32(sDO);
             // S^T(i) = K Q_i^T into the S columns (once Q_i has landed)
             auto issue_s = [&](int i) -> bool {
                 if (!mbar_wait(&bars->q_full[i & 1], (i >> 1) & 1, abort_flag)) return false;
@@ -250,12 +277,12 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (ok) ok = issue_s(0);
             for (int i = 0; ok && i < n_q; ++i) {
                 const unsigned aQ = q_addr(i);
-                const unsigned aDO = aQ + Cfg::kKVBytes;
                 // dP^T = V dO_i^T  (D=128: dP columns held dQ_{i-1} until the dQ warps copied it out)
+                if (!(ok = mbar_wait(&bars->do_full, i & 1, abort_flag))) break;
                 if (Cfg::kDqInDp && i > 0) {
                     if (!(ok = mbar_wait(&bars->dq_free, (i - 1) & 1, abort_flag))) break;
-                    tc_fence_after();
                 }
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     mma_ss(tmem + Cfg::colDP, kmajor_desc(aV, kk), kmajor_desc(aDO, kk), idesc_t, kk > 0);
@@ -267,6 +294,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int kk = 0; kk < kTile / 16; ++kk)
                     mma_ts(tmem + Cfg::colDV, tmem + Cfg::colS + packed_col(kk), mnmajor_desc(aDO, kk), idesc_g,
                            (i > 0 || kk > 0));
+                mma_commit(&bars->do_empty);           // dO_i read by dP^T(i) and dV(i)
                 if (i + 1 < n_q && !(ok = issue_s(i + 1))) break;
                 // dK += dS^T Q_i ; dQ_i^T = K^T dS^T
                 if (!(ok = mbar_wait(&bars->ds_ready, i & 1, abort_flag))) break;
@@ -328,8 +356,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         auto do_ds = [&](int t) -> bool {
             const float* dl = s_delta + (t & 1) * kTile + 64 * g;
             if (!mbar_wait(&bars->dp_full, t & 1, abort_flag)) return false;
-            // the dQ warps staged dQ_{t-1} in the dS buffer until this phase
-            if (t > 0 && !mbar_wait(&bars->sds_free, (t - 1) & 1, abort_flag)) return false;
+            // dp_full(t) was committed after dQ(t-1), so the dS buffer is free again
             tc_fence_after();
             // dS^T (keys x queries) in shared memory: MN-major operand, query block g,
             // row = key, 16-byte chunk c of the 128-byte row swizzled by (key mod 8).
@@ -405,7 +432,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int j = threadIdx.x - 384;               // 0..127
         const float* lse_h = lse + (size_t)bh * Nq;
         const float* delta_h = delta + (size_t)bh * Nq;
-        float* stage = reinterpret_cast<float*>(sDS + sub * 8192);   // this warp: 64 rows x 32 floats
+        float* stage = reinterpret_cast<float*>(sStage + sub * 8192);   // this warp: 64 rows x 32 floats
         auto stage_stats = [&](int t) {
             const int row = t * kTile + j;
             s_lse2[(t & 1) * kTile + j] = (row < Nq) ? lse_h[row] * kLog2e : INFINITY;
@@ -451,7 +478,6 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             staging_reusable();
             stage_and_reduce(v, t * kTile + 64);
             staging_reusable();
-            if (lane == 0) mbar_arrive(&bars->sds_free);   // the dS buffer is free for dS(t+1)
         }
         if (lane == 0) bulk_wait_all();                // every reduce-add has completed
     }
