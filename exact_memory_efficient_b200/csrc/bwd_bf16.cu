@@ -131,12 +131,6 @@ struct BwdBarriers {
     int abort_flag;
 };
 
-__device__ __forceinline__ uint64_t kmajor_desc(unsigned base, int kk) {
-    return make_sdesc_sw128(base + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
-}
-__device__ __forceinline__ uint64_t mnmajor_desc(unsigned base, int kk) {
-    return make_sdesc_sw128(base + kk * 16 * 128, 128 * 128, 1024);
-}
 // bf16 A operand packed in TMEM by the two compute warpgroups: query half g
 // occupies columns [64 g, 64 g + 32) of its region.
 __device__ __forceinline__ unsigned packed_col(int kk) { return (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8; }
@@ -252,22 +246,32 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
+        // Descriptors are built once and stepped by 32-bit adds of compile-time
+        // offsets, so the issuing thread keeps the tensor pipe fed.
         if (lane == 0) {
             constexpr unsigned idesc_t = make_idesc_bf16(128, 128, 0, 0);   // S^T, dP^T
             constexpr unsigned idesc_g = make_idesc_bf16(128, D, 0, 1);     // dV, dK (A in TMEM)
             constexpr unsigned idesc_q = make_idesc_bf16(128, 128, 1, 1);   // dQ^T (A = K^T, B = dS^T, MN-major)
-            const unsigned aK = smem_u32(sK), aV = smem_u32(sV), aDS = smem_u32(sDS);
+            const uint32_t k_lo = desc_lo_kmajor(smem_u32(sK));             // K as A of S^T
+            const uint32_t kt_lo = desc_lo_mnmajor(smem_u32(sK));           // K^T as A of dQ^T
+            const uint32_t v_lo = desc_lo_kmajor(smem_u32(sV));
+            const uint32_t ds_lo = desc_lo_mnmajor(smem_u32(sDS));
+            const uint32_t do_k_lo = desc_lo_kmajor(smem_u32(sDO));         // dO as B of dP^T
+            const uint32_t do_mn_lo = desc_lo_mnmajor(smem_u32(sDO));       // dO as B of dV
+            const uint32_t q_k_lo0 = desc_lo_kmajor(smem_u32(sQ));
+            const uint32_t q_mn_lo0 = desc_lo_mnmajor(smem_u32(sQ));
+            constexpr uint32_t kQStep = Cfg::kKVBytes >> 4;                  // start-field step between Q stages
+            const unsigned tS = tmem + Cfg::colS, tDP = tmem + Cfg::colDP, tDV = tmem + Cfg::colDV,
+                           tDK = tmem + Cfg::colDK, tDQ = tmem + Cfg::colDQ;
             bool ok = mbar_wait(&bars->kv_full, 0, abort_flag);
-            auto q_addr = [&](int i) -> unsigned { return smem_u32(sQ + (i & 1) * Cfg::kKVBytes); };
-            const unsigned aDO = smem_u32(sDO);
             // S^T(i) = K Q_i^T into the S columns (once Q_i has landed)
             auto issue_s = [&](int i) -> bool {
                 if (!mbar_wait(&bars->q_full[i & 1], (i >> 1) & 1, abort_flag)) return false;
                 tc_fence_after();
-                const unsigned aQ = q_addr(i);
+                const uint32_t q_lo = q_k_lo0 + (uint32_t)(i & 1) * kQStep;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    mma_ss(tmem + Cfg::colS, kmajor_desc(aK, kk), kmajor_desc(aQ, kk), idesc_t, kk > 0);
+                    mma_ss_lo(tS, k_lo + kmajor_step(kk), q_lo + kmajor_step(kk), idesc_t, kk > 0);
                 mma_commit(&bars->s_full);
                 return true;
             };
@@ -276,7 +280,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // so the compute warps form P(i+1) while dK(i) and dQ(i) run.
             if (ok) ok = issue_s(0);
             for (int i = 0; ok && i < n_q; ++i) {
-                const unsigned aQ = q_addr(i);
+                const uint32_t q_mn_lo = q_mn_lo0 + (uint32_t)(i & 1) * kQStep;
+                const unsigned acc0 = i > 0 ? 1u : 0u;
                 // dP^T = V dO_i^T  (D=128: dP columns held dQ_{i-1} until the dQ warps copied it out)
                 if (!(ok = mbar_wait(&bars->do_full, i & 1, abort_flag))) break;
                 if (Cfg::kDqInDp && i > 0) {
@@ -285,15 +290,14 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    mma_ss(tmem + Cfg::colDP, kmajor_desc(aV, kk), kmajor_desc(aDO, kk), idesc_t, kk > 0);
+                    mma_ss_lo(tDP, v_lo + kmajor_step(kk), do_k_lo + kmajor_step(kk), idesc_t, kk > 0);
                 mma_commit(&bars->dp_full);
                 // dV += P^T dO_i
                 if (!(ok = mbar_wait(&bars->p_ready, i & 1, abort_flag))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk)
-                    mma_ts(tmem + Cfg::colDV, tmem + Cfg::colS + packed_col(kk), mnmajor_desc(aDO, kk), idesc_g,
-                           (i > 0 || kk > 0));
+                    mma_ts_lo(tDV, tS + packed_col(kk), do_mn_lo + mnmajor_step(kk), idesc_g, (acc0 | kk) ? 1u : 0u);
                 mma_commit(&bars->do_empty);           // dO_i read by dP^T(i) and dV(i)
                 if (i + 1 < n_q && !(ok = issue_s(i + 1))) break;
                 // dK += dS^T Q_i ; dQ_i^T = K^T dS^T
@@ -301,15 +305,14 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk)
-                    mma_ts(tmem + Cfg::colDK, tmem + Cfg::colDP + packed_col(kk), mnmajor_desc(aQ, kk), idesc_g,
-                           (i > 0 || kk > 0));
+                    mma_ts_lo(tDK, tDP + packed_col(kk), q_mn_lo + mnmajor_step(kk), idesc_g, (acc0 | kk) ? 1u : 0u);
                 if (!Cfg::kDqInDp && i > 0) {
                     if (!(ok = mbar_wait(&bars->dq_free, (i - 1) & 1, abort_flag))) break;
                     tc_fence_after();
                 }
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk)
-                    mma_ss(tmem + Cfg::colDQ, mnmajor_desc(aK, kk), mnmajor_desc(aDS, kk), idesc_q, kk > 0);
+                    mma_ss_lo(tDQ, kt_lo + mnmajor_step(kk), ds_lo + mnmajor_step(kk), idesc_q, kk > 0);
                 mma_commit(&bars->dq_full);
                 mma_commit(&bars->q_empty[i & 1]);
             }

@@ -67,18 +67,6 @@ struct FwdBarriers {
     int abort_flag;
 };
 
-// K-major operand stored as 64-column boxes of 128 rows (128-byte swizzle):
-// descriptor for the 16-column K slice kk.
-__device__ __forceinline__ uint64_t kmajor_desc(unsigned base, int kk) {
-    return make_sdesc_sw128(base + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
-}
-
-// MN-major operand (rows = contraction index, 64-column boxes along N):
-// descriptor for rows [16 kk, 16 kk + 16).
-__device__ __forceinline__ uint64_t mnmajor_desc(unsigned base, int kk) {
-    return make_sdesc_sw128(base + kk * 16 * 128, 128 * 128, 1024);
-}
-
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -156,58 +144,76 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
+        // The issuing thread does as little as possible between tcgen05.mma
+        // instructions: descriptors are built once and stepped by 32-bit adds
+        // of compile-time offsets; ring stages are tracked incrementally.
         if (lane == 0) {
             constexpr unsigned idesc_s = make_idesc_bf16(128, kTileN, 0, 0);
             constexpr unsigned idesc_o = make_idesc_bf16(128, D, 0, 1);
-            const unsigned sQ0 = smem_u32(sQ);
-            const unsigned tS[2] = {tmem + 0u, tmem + 128u};
-            const unsigned tO[2] = {tmem + 256u, tmem + 384u};
+            const uint32_t q_lo0 = desc_lo_kmajor(smem_u32(sQ));
+            const uint32_t q_lo1 = desc_lo_kmajor(smem_u32(sQ + Cfg::kQBytes));
+            const uint32_t ring_k_lo = desc_lo_kmajor(smem_u32(sRing));
+            const uint32_t ring_v_lo = desc_lo_mnmajor(smem_u32(sRing));
+            constexpr uint32_t kStageStep = Cfg::kTileBytes >> 4;   // start-field step between ring stages
+            const unsigned tS0 = tmem, tS1 = tmem + 128u, tO0 = tmem + 256u, tO1 = tmem + 384u;
             bool ok = mbar_wait(&bars->q_full, 0, abort_flag);
-            int c = 0;  // ring tile counter
-            auto wait_full = [&](int cc) -> bool {
-                return mbar_wait(&bars->full[cc % Cfg::kStages], (cc / Cfg::kStages) & 1, abort_flag);
+            int stage = 0;
+            unsigned phase = 0;
+            // consume one ring tile: wait until it landed, return its stage offset (16-byte units)
+            auto next_tile = [&](uint32_t& off, int& st_used) -> bool {
+                if (!mbar_wait(&bars->full[stage], phase, abort_flag)) return false;
+                off = (uint32_t)stage * kStageStep;
+                st_used = stage;
+                if (++stage == Cfg::kStages) { stage = 0; phase ^= 1u; }
+                return true;
             };
-            auto ring_addr = [&](int cc) -> unsigned {
-                return smem_u32(sRing + (cc % Cfg::kStages) * Cfg::kTileBytes);
-            };
-            auto issue_s = [&](int t, unsigned kaddr) {
+            auto issue_s = [&](unsigned tS, uint32_t q_lo, uint32_t k_off) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    mma_ss(tS[t], kmajor_desc(sQ0 + t * Cfg::kQBytes, kk), kmajor_desc(kaddr, kk), idesc_s,
-                           kk > 0 ? 1u : 0u);
-                mma_commit(&bars->s_full[t]);
+                    mma_ss_lo(tS, q_lo + kmajor_step(kk), ring_k_lo + k_off + kmajor_step(kk), idesc_s, kk > 0);
             };
-            if (ok) ok = wait_full(c);
+            auto issue_pv = [&](unsigned tO, unsigned tS, uint32_t v_off, unsigned acc0) {
+#pragma unroll
+                for (int kk = 0; kk < kTileN / 16; ++kk)
+                    mma_ts_lo(tO, tS + kk * 8, ring_v_lo + v_off + mnmajor_step(kk), idesc_o, (acc0 | kk) ? 1u : 0u);
+            };
+            uint32_t k_off = 0;
+            int k_stage = 0;
+            if (ok) ok = next_tile(k_off, k_stage);
             if (ok) {
                 tc_fence_after();
-                const unsigned k0 = ring_addr(c);
-                issue_s(0, k0);
-                issue_s(1, k0);
-                mma_commit(&bars->empty[c % Cfg::kStages]);
-                ++c;
+                issue_s(tS0, q_lo0, k_off);
+                mma_commit(&bars->s_full[0]);
+                issue_s(tS1, q_lo1, k_off);
+                mma_commit(&bars->s_full[1]);
+                mma_commit(&bars->empty[k_stage]);
             }
             for (int j = 0; ok && j < n_kv; ++j) {
-                const int cv = c;          // V_j
-                const int ck = c + 1;      // K_{j+1}
                 const bool more = (j + 1 < n_kv);
-                if (!(ok = wait_full(cv))) break;
-                const unsigned vaddr = ring_addr(cv);
-                for (int t = 0; t < 2; ++t) {
-                    if (!(ok = mbar_wait(&bars->p_ready[t], j & 1, abort_flag))) break;
+                const unsigned acc0 = j > 0 ? 1u : 0u;
+                uint32_t v_off = 0;
+                int v_stage = 0;
+                if (!(ok = next_tile(v_off, v_stage))) break;
+                // tile 0: O_0 += P_0 V_j, then S_0 = Q_0 K_{j+1}^T
+                if (!(ok = mbar_wait(&bars->p_ready[0], j & 1, abort_flag))) break;
+                tc_fence_after();
+                issue_pv(tO0, tS0, v_off, acc0);
+                if (more) {
+                    if (!(ok = next_tile(k_off, k_stage))) break;
                     tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < kTileN / 16; ++kk)
-                        mma_ts(tO[t], tS[t] + kk * 8, mnmajor_desc(vaddr, kk), idesc_o,
-                               (j > 0 || kk > 0) ? 1u : 0u);
-                    if (t == 1) mma_commit(&bars->empty[cv % Cfg::kStages]);
-                    if (more) {
-                        if (t == 0 && !(ok = wait_full(ck))) break;
-                        tc_fence_after();
-                        issue_s(t, ring_addr(ck));
-                        if (t == 1) mma_commit(&bars->empty[ck % Cfg::kStages]);
-                    }
+                    issue_s(tS0, q_lo0, k_off);
+                    mma_commit(&bars->s_full[0]);
                 }
-                c += 2;
+                // tile 1: O_1 += P_1 V_j, then S_1 = Q_1 K_{j+1}^T
+                if (!(ok = mbar_wait(&bars->p_ready[1], j & 1, abort_flag))) break;
+                tc_fence_after();
+                issue_pv(tO1, tS1, v_off, acc0);
+                mma_commit(&bars->empty[v_stage]);
+                if (more) {
+                    issue_s(tS1, q_lo1, k_off);
+                    mma_commit(&bars->s_full[1]);
+                    mma_commit(&bars->empty[k_stage]);
+                }
             }
             if (ok) mma_commit(&bars->o_final);
             // drain: every MMA issued above has completed before TMEM is freed

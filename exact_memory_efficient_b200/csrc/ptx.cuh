@@ -266,6 +266,51 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(unsigned smem_addr, unsigne
     return d;
 }
 
+// The same descriptor as two 32-bit words.  Every operand here is 128-byte
+// swizzled with SBO = 1024, so the high word is one constant; the low word
+// holds the start address (addr >> 4, bits 0-13) and the LBO field (bits
+// 16-29).  Stepping through a tile only changes the start field, so a K step is
+// a single 32-bit add of (byte offset >> 4): the start field cannot carry out
+// of its 14 bits because shared memory addresses stay below 256 KB.  Keeping
+// this arithmetic to one add matters: the one thread that issues MMAs runs
+// them back to back, and a dependent chain of 64-bit descriptor math before
+// each tcgen05.mma halves the tensor pipe's throughput.
+constexpr uint32_t kDescHiSw128 = (1024u >> 4) | (1u << 14) | (2u << 29);
+// K-major operand (K contiguous in 128-byte rows; LBO unused = 16 bytes).
+__device__ __forceinline__ uint32_t desc_lo_kmajor(unsigned smem_addr) { return (smem_addr >> 4) | (1u << 16); }
+// MN-major operand (64-element blocks along M/N 16 KB apart: LBO = 16384).
+__device__ __forceinline__ uint32_t desc_lo_mnmajor(unsigned smem_addr) {
+    return (smem_addr >> 4) | ((16384u >> 4) << 16);
+}
+// Start-field offset of K step kk (16 elements): K-major tiles are stored as
+// 64-column boxes of 128 rows (16 KB), MN-major tiles advance 16 rows of 128 B.
+__host__ __device__ constexpr uint32_t kmajor_step(int kk) { return (kk >> 2) * 1024u + (kk & 3) * 2u; }
+__host__ __device__ constexpr uint32_t mnmajor_step(int kk) { return kk * 128u; }
+
+// D[tmem] (+)= A[smem] * B[smem]^T with descriptors given by their low words.
+__device__ __forceinline__ void mma_ss_lo(unsigned d_tmem, uint32_t a_lo, uint32_t b_lo, unsigned idesc,
+                                          unsigned accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+        "mov.b64 da, {%1, %3};\n\t"
+        "mov.b64 db, {%2, %3};\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(kDescHiSw128), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]^T with the B descriptor given by its low word.
+__device__ __forceinline__ void mma_ts_lo(unsigned d_tmem, unsigned a_tmem, uint32_t b_lo, unsigned idesc,
+                                          unsigned accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+        "mov.b64 db, {%2, %3};\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "r"(b_lo), "r"(kDescHiSw128), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
 //   bits 4-5 D format (1 = f32); 7-9 A format (1 = bf16); 10-12 B format (1 = bf16)
 //   bit 15 A major (0 = K, 1 = MN); bit 16 B major; bits 17-22 N >> 3; bits 24-28 M >> 4
