@@ -246,9 +246,17 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int c = 0; c < kTileN; ++c)
                     if (c >= nvalid) sr[c] = __float_as_uint(-INFINITY);
             }
-            float mx = __uint_as_float(sr[0]);
+            // row maximum as 8 independent chains (one thread owns the row, so a
+            // single 128-long dependent chain would dominate the softmax latency)
+            float mxa[8];
 #pragma unroll
-            for (int c = 1; c < kTileN; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
+            for (int i = 0; i < 8; ++i) mxa[i] = __uint_as_float(sr[i]);
+#pragma unroll
+            for (int c = 8; c < kTileN; c += 8)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mxa[i] = fmaxf(mxa[i], __uint_as_float(sr[c + i]));
+            const float mx = fmaxf(fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])),
+                                   fmaxf(fmaxf(mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7])));
             const float m_blk = mx * c_log2;
             float m_new = m_ref;
             bool rescale = false;
@@ -263,7 +271,10 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             m_ref = m_new;
             l *= alpha;
-            float rowsum = 0.f;
+            // row sum as 8 independent partial sums (same reason as the maximum)
+            float rsa[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) rsa[i] = 0.f;
 #pragma unroll
             for (int c0 = 0; c0 < kTileN; c0 += 32) {
                 uint32_t pk[16];
@@ -271,12 +282,12 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int c = 0; c < 32; c += 2) {
                     const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c0 + c]), c_log2, -m_ref));
                     const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c0 + c + 1]), c_log2, -m_ref));
-                    rowsum += p0 + p1;
+                    rsa[(c / 2) & 7] += p0 + p1;
                     pk[c / 2] = pack_bf16x2(p0, p1);
                 }
                 tmem_st16(tS + c0 / 2, pk);
             }
-            l += rowsum;
+            l += ((rsa[0] + rsa[1]) + (rsa[2] + rsa[3])) + ((rsa[4] + rsa[5]) + (rsa[6] + rsa[7]));
             if (rescale) {
                 // PV_t(j-1) has completed (it was issued before S_t(j), whose
                 // commit we waited on), so O_t can be rescaled in place.
