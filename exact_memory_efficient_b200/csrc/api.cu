@@ -222,6 +222,17 @@ mea_status_t mea_attn_fwd(const void* q, const void* k, const void* v, void* o, 
     a.D = D;
     a.scale = scale;
     if (BH > 65535) return MEA_ERR_UNSUPPORTED;
+    // Split the keys over a cluster when the (query tile x head) grid would
+    // leave most SMs idle, e.g. decode-shaped calls with a handful of rows.
+    {
+        const long long base = (long long)((Nq + 255) / 256) * BH;
+        const int key_tiles = (Nk + 127) / 128;
+        int chunks = 1;
+        while (chunks < 16 && base * chunks * 2 <= dev->sm_count && key_tiles >= chunks * 4) chunks *= 2;
+        a.chunks = chunks;
+        a.chunk_len = (int)round_up((size_t)((Nk + chunks - 1) / chunks), 128);
+        if ((long long)((Nq + 255) / 256) * chunks > 0x7fffffffLL) return MEA_ERR_UNSUPPORTED;
+    }
     return cuda_status(mea::launch_fwd_bf16(a, s), "fwd_bf16 launch");
 }
 

@@ -22,12 +22,21 @@
 //               maximum moves.
 // TMEM (512 columns): S_0 [0,128)  S_1 [128,256)  O_0 [256,256+D)  O_1 [384,384+D).
 //
+// Key split (decode-shaped calls): when a grid would leave most SMs idle (few
+// query tiles x heads), the keys of each (batch, head, query tile) are split
+// over the CTAs of a thread-block cluster.  Each CTA runs the recurrence over
+// its chunk and leaves the chunk summary of every row -- its reference maximum,
+// exp-sum and unnormalised accumulator -- in its shared memory; the cluster's
+// first CTA merges the summaries through distributed shared memory with the
+// two-block formulas and writes O and lse.  No global scratch is used.
+//
 // Reference maximum: a row's exponentials are taken relative to a reference
 // value m_ref that is raised to the true running maximum only when the new
 // block maximum exceeds it by more than 8 (base-2 units).  Then every
 // exponential is <= 2^8, nothing overflows, and because O, l and the final
 // lse all use the same m_ref the result is the same exact softmax; it only
 // saves O rescales.
+#include <cooperative_groups.h>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -67,15 +76,35 @@ struct FwdBarriers {
     int abort_flag;
 };
 
+// Chunk summaries for the cluster merge live where Q and the K/V ring were
+// (free once the last MMA has completed): rows of D floats padded to D + 4 so
+// that one row per lane is written without shared-memory bank conflicts.
+template <int D>
+__device__ __forceinline__ float* part_row(uint8_t* smem, int t, int r) {
+    return reinterpret_cast<float*>(smem) + ((size_t)t * kTileM + r) * (D + 4);
+}
+template <int D>
+__device__ __forceinline__ float* part_ml(uint8_t* smem, int t, int r) {
+    return reinterpret_cast<float*>(smem) + (size_t)2 * kTileM * (D + 4) + ((size_t)t * kTileM + r) * 2;
+}
+static_assert(2 * 128 * (128 + 4) * 4 + 2 * 128 * 2 * 4 <= FwdCfg<128>::kSmemData, "merge area (D=128)");
+static_assert(2 * 128 * (64 + 4) * 4 + 2 * 128 * 2 * 4 <= FwdCfg<64>::kSmemData, "merge area (D=64)");
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ o,
-                float* __restrict__ lse, int Nq, int Nk, float scale) {
+                float* __restrict__ lse, int Nq, int Nk, float scale, int chunk_len) {
     using Cfg = FwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
-    // 1024-byte alignment for the 128-byte-swizzle atoms
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte alignment of the shared-memory address (not of the generic
+    // pointer: in a cluster launch each CTA's shared window can sit at a
+    // different generic offset) for the 128-byte-swizzle atoms
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* sQ = smem;                               // Q_0 then Q_1
     uint8_t* sRing = smem + 2 * Cfg::kQBytes;         // kStages tiles
     FwdBarriers* bars = reinterpret_cast<FwdBarriers*>(smem + Cfg::kSmemData);
@@ -83,8 +112,14 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const unsigned warp = warp_id();
     const unsigned lane = lane_id();
     const int bh = blockIdx.y;
-    const int m0 = blockIdx.x * (2 * kTileM);
-    const int n_kv = (Nk + kTileN - 1) / kTileN;
+    // key split over the CTAs of a cluster (one CTA per cluster when not split)
+    unsigned nranks, rank;
+    asm("mov.u32 %0, %%cluster_nctarank;" : "=r"(nranks));
+    asm("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
+    const int m0 = (blockIdx.x / nranks) * (2 * kTileM);
+    const int c_begin = (nranks > 1) ? (int)rank * chunk_len : 0;
+    const int c_end = (nranks > 1) ? min(Nk, c_begin + chunk_len) : Nk;
+    const int n_kv = (c_end > c_begin) ? (c_end - c_begin + kTileN - 1) / kTileN : 0;
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 1);
@@ -131,7 +166,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 uint8_t* dst = sRing + s * Cfg::kTileBytes;
                 const CUtensorMap* tm = (c & 1) ? &tm_v : &tm_k;
-                const int key0 = (c >> 1) * kTileN;
+                const int key0 = c_begin + (c >> 1) * kTileN;
                 mbar_arrive_expect_tx(&bars->full[s], Cfg::kTileBytes);
                 for (int b = 0; b < D / 64; ++b)
                     tma_load_3d(dst + b * Cfg::kBoxBytes, tm, &bars->full[s], b * 64, key0, bh);
@@ -172,15 +207,33 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int kk = 0; kk < D / 16; ++kk)
                     mma_ss_lo(tS, q_lo + kmajor_step(kk), ring_k_lo + k_off + kmajor_step(kk), idesc_s, kk > 0);
             };
+            // In a cluster launch (key split) P V is issued per 64-column block of V,
+            // each block addressed by its start address: on this part, an MMA on
+            // a CTA of cluster rank 1 read the second 64-element block of an
+            // MN-major B operand wrongly when reaching it through the
+            // descriptor's leading-byte offset (rank 0 and non-cluster launches
+            // were correct).  The single N = D instruction is kept otherwise.
+            const bool pv_by_block = (D > 64) && (nranks > 1);
             auto issue_pv = [&](unsigned tO, unsigned tS, uint32_t v_off, unsigned acc0) {
+                if (pv_by_block) {
+                    constexpr unsigned idesc_o64 = make_idesc_bf16(128, 64, 0, 1);
 #pragma unroll
-                for (int kk = 0; kk < kTileN / 16; ++kk)
-                    mma_ts_lo(tO, tS + kk * 8, ring_v_lo + v_off + mnmajor_step(kk), idesc_o, (acc0 | kk) ? 1u : 0u);
+                    for (int blk = 0; blk < D / 64; ++blk)
+#pragma unroll
+                        for (int kk = 0; kk < kTileN / 16; ++kk)
+                            mma_ts_lo(tO + 64 * blk, tS + kk * 8,
+                                      ring_v_lo + v_off + blk * (Cfg::kBoxBytes >> 4) + mnmajor_step(kk), idesc_o64,
+                                      (acc0 | kk) ? 1u : 0u);
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < kTileN / 16; ++kk)
+                        mma_ts_lo(tO, tS + kk * 8, ring_v_lo + v_off + mnmajor_step(kk), idesc_o, (acc0 | kk) ? 1u : 0u);
+                }
             };
             uint32_t k_off = 0;
             int k_stage = 0;
-            if (ok) ok = next_tile(k_off, k_stage);
-            if (ok) {
+            if (ok && n_kv > 0) ok = next_tile(k_off, k_stage);
+            if (ok && n_kv > 0) {
                 tc_fence_after();
                 issue_s(tS0, q_lo0, k_off);
                 mma_commit(&bars->s_full[0]);
@@ -240,7 +293,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int c0 = 0; c0 < kTileN; c0 += 32)
                 tmem_ld32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(&sr[c0]));
             tmem_wait_ld();
-            const int nvalid = Nk - j * kTileN;
+            const int nvalid = c_end - (c_begin + j * kTileN);
             if (nvalid < kTileN) {
 #pragma unroll
                 for (int c = 0; c < kTileN; ++c)
@@ -308,27 +361,106 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (ok && mbar_wait(&bars->o_final, 0, abort_flag)) {
             tc_fence_after();
             const int row = m0 + t * kTileM + r;
-            const float inv_l = 1.f / l;
-            uint16_t* orow = o + ((size_t)bh * Nq + row) * D;
+            if (nranks == 1) {
+                const float inv_l = 1.f / l;
+                uint16_t* orow = o + ((size_t)bh * Nq + row) * D;
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t ov[32];
-                tmem_ld32(tO + c0, ov);
-                tmem_wait_ld();
-                if (row < Nq) {
-                    uint32_t packed[16];
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t ov[32];
+                    tmem_ld32(tO + c0, ov);
+                    tmem_wait_ld();
+                    if (row < Nq) {
+                        uint32_t packed[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        packed[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l,
-                                                __uint_as_float(ov[2 * i + 1]) * inv_l);
-                    uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+                        for (int i = 0; i < 16; ++i)
+                            packed[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l,
+                                                    __uint_as_float(ov[2 * i + 1]) * inv_l);
+                        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                    }
                 }
+                if (row < Nq) lse[(size_t)bh * Nq + row] = (m_ref + __log2f(l)) * kLn2;
+            } else {
+                // chunk summary of this row for the cluster merge: (m_ref, l) and the
+                // unnormalised accumulator (zero when this CTA's chunk is empty)
+                float* prow = part_row<D>(smem, t, r);
+#pragma unroll
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t ov[32];
+                    tmem_ld32(tO + c0, ov);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        float4 f = (n_kv > 0) ? make_float4(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1]),
+                                                            __uint_as_float(ov[i + 2]), __uint_as_float(ov[i + 3]))
+                                              : make_float4(0.f, 0.f, 0.f, 0.f);
+                        *reinterpret_cast<float4*>(prow + c0 + i) = f;
+                    }
+                }
+                float* ml = part_ml<D>(smem, t, r);
+                ml[0] = (n_kv > 0) ? m_ref : -INFINITY;
+                ml[1] = (n_kv > 0) ? l : 0.f;
             }
-            if (row < Nq) lse[(size_t)bh * Nq + row] = (m_ref + __log2f(l)) * kLn2;
         }
+    }
+
+    if (nranks > 1) {
+        // every thread of every CTA of the cluster passes both barriers, also
+        // on the abort path, so no CTA leaves while another reads its memory
+        __syncwarp();
+        cluster_sync_all();
+        if (rank == 0 && warp >= 2) {
+            namespace cg = cooperative_groups;
+            cg::cluster_group cluster = cg::this_cluster();
+            const int t = (warp - 2) >> 2;
+            const int r = (warp & 3) * 32 + lane;
+            const int row = m0 + t * kTileM + r;
+            if (row < Nq && !*abort_flag) {
+                float M = -INFINITY;
+                for (unsigned c = 0; c < nranks; ++c) {
+                    const float* ml = cluster.map_shared_rank(part_ml<D>(smem, t, r), c);
+                    M = fmaxf(M, ml[0]);
+                }
+                float L = 0.f;
+                float w[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    w[c] = 0.f;
+                    if (c < (int)nranks) {
+                        const float* ml = cluster.map_shared_rank(part_ml<D>(smem, t, r), (unsigned)c);
+                        w[c] = ex2_approx(ml[0] - M);     // 0 for empty chunks (m = -inf)
+                        L = fmaf(w[c], ml[1], L);
+                    }
+                }
+                const float inv_L = 1.f / L;
+                uint16_t* orow = o + ((size_t)bh * Nq + row) * D;
+#pragma unroll 1
+                for (int d = 0; d < D; d += 8) {
+                    float acc[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        if (c < (int)nranks) {
+                            const float* prow = cluster.map_shared_rank(part_row<D>(smem, t, r), (unsigned)c);
+                            const float4 a = *reinterpret_cast<const float4*>(prow + d);
+                            const float4 b = *reinterpret_cast<const float4*>(prow + d + 4);
+                            acc[0] = fmaf(w[c], a.x, acc[0]); acc[1] = fmaf(w[c], a.y, acc[1]);
+                            acc[2] = fmaf(w[c], a.z, acc[2]); acc[3] = fmaf(w[c], a.w, acc[3]);
+                            acc[4] = fmaf(w[c], b.x, acc[4]); acc[5] = fmaf(w[c], b.y, acc[5]);
+                            acc[6] = fmaf(w[c], b.z, acc[6]); acc[7] = fmaf(w[c], b.w, acc[7]);
+                        }
+                    }
+                    *reinterpret_cast<uint4*>(orow + d) =
+                        make_uint4(pack_bf16x2(acc[0] * inv_L, acc[1] * inv_L), pack_bf16x2(acc[2] * inv_L, acc[3] * inv_L),
+                                   pack_bf16x2(acc[4] * inv_L, acc[5] * inv_L), pack_bf16x2(acc[6] * inv_L, acc[7] * inv_L));
+                }
+                lse[(size_t)bh * Nq + row] = (M + __log2f(L)) * kLn2;
+            }
+        }
+        cluster_sync_all();
     }
 
     tc_fence_before();
@@ -345,9 +477,29 @@ cudaError_t launch_d(const Bf16FwdArgs& a, cudaStream_t stream) {
     auto kern = fwd_bf16_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
-    dim3 grid((a.Nq + 2 * kTileM - 1) / (2 * kTileM), a.BH, 1);
-    kern<<<grid, kThreads, Cfg::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.o, a.lse, a.Nq, a.Nk, a.scale);
-    return cudaGetLastError();
+    const int q_tiles = (a.Nq + 2 * kTileM - 1) / (2 * kTileM);
+    if (a.chunks <= 1) {
+        dim3 grid(q_tiles, a.BH, 1);
+        kern<<<grid, kThreads, Cfg::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.o, a.lse, a.Nq, a.Nk, a.scale, 0);
+        return cudaGetLastError();
+    }
+    if (a.chunks > 8) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(q_tiles * a.chunks, a.BH, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = a.chunks;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a.tm_q, a.tm_k, a.tm_v, a.o, a.lse, a.Nq, a.Nk, a.scale, a.chunk_len);
 }
 
 }  // namespace

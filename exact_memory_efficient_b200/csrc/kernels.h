@@ -33,6 +33,8 @@ struct Bf16FwdArgs {
     float* lse;
     int BH, Nq, Nk, D;
     float scale;
+    int chunks;     // CTAs per cluster splitting the keys (1 = no split)
+    int chunk_len;  // keys per chunk (multiple of 128) when chunks > 1
 };
 cudaError_t launch_fwd_bf16(const Bf16FwdArgs& a, cudaStream_t stream);
 

@@ -50,6 +50,19 @@ def test_shapes_full(B, H, Nq, Nk, D):
     full_check(q, k, v, w.scale, f"{(B, H, Nq, Nk, D)}", bf16_output=True)
 
 
+@pytest.mark.parametrize("B,H,Nq,Nk,D", [
+    (1, 8, 1, 16384, 128),    # decode: 16 chunks of 1024 keys over a cluster, merged in distributed smem
+    (2, 4, 3, 5000, 64),      # 16 chunks of 384 keys: one of 8 keys, the last two empty
+    (1, 2, 200, 2049, 128),   # 8 chunks of 384 keys: one of 129 keys, the last two empty
+    (1, 1, 1, 8193, 128),     # 16 chunks of 640 keys: one of 513 keys, the last three empty
+    (1, 3, 257, 1024, 64),    # two query tiles per CTA, 4 chunks of 256 keys
+])
+def test_decode_key_split(B, H, Nq, Nk, D):
+    w = custom(B, H, Nq, Nk, D, "bf16", backward=False)
+    q, k, v, _ = make_inputs(w, 17)
+    full_check(q, k, v, w.scale, f"{(B, H, Nq, Nk, D)}", bf16_output=True)
+
+
 @pytest.mark.parametrize("seed", [0, 1, 2])
 def test_encoder_512_full(seed):
     w = make_workload("encoder_512_bf16")
