@@ -324,24 +324,30 @@ def run_ours(args):
                                                "main": round(main_avg_ms, 4),
                                                "finalize": round(statistics.mean(fin_ms), 4)}}
     if rank == 0 and not args.no_extras:
-        ws1 = make_workload("single_query_f32")
-        q1, k1, v1, _ = (x.to(dev) if x is not None else None for x in make_inputs(ws1, 0))
-        o1, l1 = m.attention_forward(q1, k1, v1, ws1.scale)
-        for _ in range(5):
-            m.mea_attn_fwd(q1, k1, v1, o1, l1, ws1.scale)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = 50
-        e0.record(stream)
-        for _ in range(reps):
-            m.mea_attn_fwd(q1, k1, v1, o1, l1, ws1.scale)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        us = e0.elapsed_time(e1) * 1e3 / reps
-        byts = (q1.numel() + k1.numel() + v1.numel() + o1.numel() + l1.numel()) * 4
-        rows["single_query_f32_fwd"] = {"us": round(us, 2), "GB/s": round(byts / (us * 1e-6) / 1e9, 1),
-                                        "frac_of_hbm": round(byts / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 3),
-                                        "note": "L2-warm back-to-back launches (67 MB working set < L2)"}
-        del q1, k1, v1, o1, l1
+        # HBM-bound decode-shaped forwards, timed one launch at a time with L2
+        # flushed in between (their K/V would otherwise stay L2-resident)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        for wname in ("single_query_f32", "decode_16384_bf16"):
+            wd = make_workload(wname)
+            qd, kd, vd, _ = (x.to(dev) if x is not None else None for x in make_inputs(wd, 0))
+            od, ld = m.attention_forward(qd, kd, vd, wd.scale)
+            for _ in range(3):
+                m.mea_attn_fwd(qd, kd, vd, od, ld, wd.scale)
+            reps = 20
+            evs_d = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+            for e0, e1 in evs_d:
+                flush.zero_()
+                e0.record(stream)
+                m.mea_attn_fwd(qd, kd, vd, od, ld, wd.scale)
+                e1.record(stream)
+            torch.cuda.synchronize()
+            us = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs_d) * 1e3
+            byts = sum(x.numel() * x.element_size() for x in (qd, kd, vd, od, ld))
+            rows[f"{wname}_fwd"] = {"us": round(us, 2), "GB/s": round(byts / (us * 1e-6) / 1e9, 1),
+                                    "frac_of_hbm": round(byts / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 3),
+                                    "bytes": byts, "note": "median of 20 launches, L2 flushed before each"}
+            del qd, kd, vd, od, ld
+        del flush
 
     # ---- extra memory versus a materialised-scores attention (arithmetic)
     naive_scores = w.B * w.H * w.Nq * w.Nk * 4

@@ -62,6 +62,8 @@ WORKLOADS = {
     "encoder_512_bf16": Workload("encoder_512_bf16", 32, 8, 512, 512, 64, "bf16", True,
                                  note="encoder-shaped batch B32 H8 N512 D64"),
 }
+WORKLOADS["decode_16384_bf16"] = Workload("decode_16384_bf16", 1, 8, 1, 16384, 128, "bf16", False,
+                                          note="decode-shaped bf16 forward: one query row over 16384 keys, 8 heads")
 for _n in (256, 1024, 4096, 16384):
     WORKLOADS[f"long_{_n}_bf16"] = Workload(f"long_{_n}_bf16", 1, 16, _n, _n, 128, "bf16", True,
                                              note=f"long-sequence sweep B1 H16 N{_n} D128")
