@@ -18,6 +18,8 @@ from .attention import (  # noqa: F401
     attention_backward_2d,
     attention_forward,
     attention_backward,
+    attention_forward_gqa,
+    attention_backward_gqa,
     attention_forward_rows,
     attention_backward_rows,
     attention_backward_keys,

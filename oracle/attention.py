@@ -119,6 +119,51 @@ def attention_backward(q, k, v, do, scale):
     return dq, dk, dv, o, lse
 
 
+# ------------------------------------------ shared key/value heads (GQA)
+#
+# "当注意力成为瓶颈从on困境到线性复杂度的技术突围", section 推理优化：减少KV Cache:
+# multi-query and grouped-query attention let several query heads share one
+# key/value head.  With H query heads and H_kv key/value heads (H a multiple of
+# H_kv), query head h reads key/value head h // (H / H_kv): the page splits the
+# query heads into consecutive groups without fixing the order, and consecutive
+# groups are the plainest reading.  A shared K/V head is a parameter used by
+# several heads, so its gradient is the sum over the heads that read it.
+
+def attention_forward_gqa(q, k, v, scale):
+    """q [B,H,Nq,D], k/v [B,H_kv,Nk,D] -> (O [B,H,Nq,D], lse [B,H,Nq])."""
+    q, k, v = _heads(q), _heads(k), _heads(v)
+    B, H, Nq, _ = q.shape
+    Hkv = k.shape[1]
+    assert H % Hkv == 0, "H must be a multiple of H_kv"
+    G = H // Hkv
+    o = np.empty((B, H, Nq, v.shape[3]))
+    lse = np.empty((B, H, Nq))
+    for b in range(B):
+        for h in range(H):
+            o[b, h], lse[b, h] = attention_forward_2d(q[b, h], k[b, h // G], v[b, h // G], scale)
+    return o, lse
+
+
+def attention_backward_gqa(q, k, v, do, scale):
+    """Gradients for shared key/value heads: dq [B,H,..], dk/dv [B,H_kv,..] summed over each group."""
+    q, k, v, do = _heads(q), _heads(k), _heads(v), _heads(do)
+    B, H = q.shape[:2]
+    Hkv = k.shape[1]
+    assert H % Hkv == 0, "H must be a multiple of H_kv"
+    G = H // Hkv
+    dq = np.empty_like(q)
+    dk, dv = np.zeros_like(k), np.zeros_like(v)
+    o = np.empty(q.shape[:3] + (v.shape[3],))
+    lse = np.empty(q.shape[:3])
+    for b in range(B):
+        for h in range(H):
+            dq[b, h], dk_h, dv_h, o[b, h], lse[b, h] = attention_backward_2d(
+                q[b, h], k[b, h // G], v[b, h // G], do[b, h], scale)
+            dk[b, h // G] += dk_h
+            dv[b, h // G] += dv_h
+    return dq, dk, dv, o, lse
+
+
 # ------------------------------------------- sampled outputs at full size
 #
 # Query rows are independent problems, so the forward of a subset of rows is the

@@ -353,3 +353,56 @@ def test_pins_catch_planted_forward_mistakes():
     s = c["scale"] * (q @ k.T)
     lse_base2 = np.log2(np.exp(s).sum(1))
     assert abs(lse_base2[0] - c["lse"][0]) > 1e-3
+
+
+# ------------------------------------------------- shared key/value heads
+
+def _loss_gqa(q, k, v, do, scale):
+    o, _ = oracle.attention_forward_gqa(q, k, v, scale)
+    return float((do * o).sum())
+
+
+@pytest.mark.parametrize("H,Hkv", [(4, 2), (3, 1), (2, 2)])
+def test_gqa_finite_differences(H, Hkv):
+    """Brute-force gradients of the shared-head loss, including the sum over each group."""
+    rng = np.random.default_rng(H * 10 + Hkv)
+    Nq, Nk, D, scale = 3, 4, 2, 0.8
+    q = rng.standard_normal((1, H, Nq, D))
+    k = rng.standard_normal((1, Hkv, Nk, D))
+    v = rng.standard_normal((1, Hkv, Nk, D))
+    do = rng.standard_normal((1, H, Nq, D))
+    dq, dk, dv, _, _ = oracle.attention_backward_gqa(q, k, v, do, scale)
+    np.testing.assert_allclose(dq, _central_diff(lambda x: _loss_gqa(x, k, v, do, scale), q), atol=1e-8)
+    np.testing.assert_allclose(dk, _central_diff(lambda x: _loss_gqa(q, x, v, do, scale), k), atol=1e-8)
+    np.testing.assert_allclose(dv, _central_diff(lambda x: _loss_gqa(q, k, x, do, scale), v), atol=1e-8)
+
+
+def test_gqa_matches_torch_autograd_with_shared_heads():
+    """torch fp64 autograd with K/V expanded by repeat_interleave (an independent library path)."""
+    g = torch.Generator().manual_seed(5)
+    B, H, Hkv, Nq, Nk, D = 2, 6, 2, 9, 13, 8
+    q = torch.randn(B, H, Nq, D, generator=g, dtype=torch.float64)
+    k = torch.randn(B, Hkv, Nk, D, generator=g, dtype=torch.float64)
+    v = torch.randn(B, Hkv, Nk, D, generator=g, dtype=torch.float64)
+    do = torch.randn(B, H, Nq, D, generator=g, dtype=torch.float64)
+    scale = 0.3
+    qt, kt, vt = (x.clone().requires_grad_(True) for x in (q, k, v))
+    ke = kt.repeat_interleave(H // Hkv, dim=1)
+    ve = vt.repeat_interleave(H // Hkv, dim=1)
+    ot = torch.matmul(torch.softmax(torch.matmul(qt, ke.transpose(-1, -2)) * scale, dim=-1), ve)
+    ot.backward(do)
+    o, lse = oracle.attention_forward_gqa(q.numpy(), k.numpy(), v.numpy(), scale)
+    np.testing.assert_allclose(o, ot.detach().numpy(), atol=1e-12)
+    dq, dk, dv, _, _ = oracle.attention_backward_gqa(q.numpy(), k.numpy(), v.numpy(), do.numpy(), scale)
+    np.testing.assert_allclose(dq, qt.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dk, kt.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dv, vt.grad.numpy(), atol=1e-11)
+
+
+def test_gqa_single_group_is_mha():
+    rng = np.random.default_rng(3)
+    q, k, v, do = (rng.standard_normal((1, 3, 5, 4)) for _ in range(4))
+    a = oracle.attention_backward_gqa(q, k, v, do, 0.5)
+    b = oracle.attention_backward(q, k, v, do, 0.5)
+    for x, y in zip(a, b):
+        np.testing.assert_allclose(x, y, atol=1e-14)
