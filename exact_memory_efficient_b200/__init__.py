@@ -9,6 +9,9 @@ to own device memory and streams.
 
     o, lse = attention_forward(q, k, v)                 # allocates o, lse
     dq, dk, dv = attention_backward(q, k, v, o, lse, do)  # allocates grads + workspace
+
+k and v may have fewer heads than q (grouped- or multi-query attention); the
+helpers then call the ``_gqa`` entry points.
 """
 
 from __future__ import annotations
@@ -24,7 +27,8 @@ __all__ = [
     "MEA_OK", "MEA_ERR_INVALID_ARG", "MEA_ERR_UNSUPPORTED", "MEA_ERR_MISALIGNED", "MEA_ERR_WORKSPACE",
     "MEA_ERR_CUDA", "MEA_ERR_TIMEOUT", "MEA_DTYPE_F32", "MEA_DTYPE_BF16",
     "MEA_BWD_ALL", "MEA_BWD_PREPROCESS", "MEA_BWD_MAIN", "MEA_BWD_FINALIZE",
-    "mea_attn_fwd", "mea_attn_bwd", "mea_attn_bwd_phase", "mea_attn_bwd_workspace_size", "mea_attn_bwd_noalloc", "mea_last_device_error",
+    "mea_attn_fwd", "mea_attn_bwd", "mea_attn_bwd_phase", "mea_attn_bwd_workspace_size", "mea_attn_bwd_noalloc",
+    "mea_attn_fwd_gqa", "mea_attn_bwd_gqa", "mea_attn_bwd_gqa_workspace_size", "mea_last_device_error",
     "mea_selftest_bounded_wait", "mea_status_string", "mea_last_error_message", "mea_version", "attention_forward", "attention_backward",
 ]
 
@@ -82,6 +86,12 @@ def load_library() -> ctypes.CDLL:
     lib.mea_attn_bwd_phase.restype = i
     lib.mea_attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     lib.mea_attn_bwd_noalloc.restype = i
+    lib.mea_attn_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
+    lib.mea_attn_fwd_gqa.restype = i
+    lib.mea_attn_bwd_gqa_workspace_size.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(sz)]
+    lib.mea_attn_bwd_gqa_workspace_size.restype = i
+    lib.mea_attn_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, sz, vp]
+    lib.mea_attn_bwd_gqa.restype = i
     lib.mea_selftest_bounded_wait.argtypes = [vp, vp]
     lib.mea_selftest_bounded_wait.restype = i
     lib.mea_last_device_error.argtypes = [vp]
@@ -199,6 +209,52 @@ def mea_attn_bwd_noalloc(q, k, v, o, lse, do, dq, dk, dv, scale: float, stream=N
     _check(st, "mea_attn_bwd_noalloc")
 
 
+def _gqa_shapes(q, k, where: str):
+    B, H, Nq, D = _bhnd(q, "q")
+    Bk, Hkv, Nk, Dk = _bhnd(k, "k")
+    if (Bk, Dk) != (B, D) or Hkv < 1 or H % Hkv != 0:
+        raise MeaError(MEA_ERR_INVALID_ARG, f"{where}: k must be [B, H_kv, Nk, D] with H a multiple of H_kv")
+    return B, H, Hkv, Nq, Nk, D
+
+
+def mea_attn_fwd_gqa(q, k, v, o, lse, scale: float, stream=None) -> None:
+    """C ``mea_attn_fwd_gqa``: q, o [B,H,Nq,D]; k, v [B,H_kv,Nk,D]; query head h reads key/value
+    head h // (H // H_kv)."""
+    B, H, Hkv, Nq, Nk, D = _gqa_shapes(q, k, "mea_attn_fwd_gqa")
+    if tuple(v.shape) != tuple(k.shape) or tuple(o.shape) != tuple(q.shape):
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_fwd_gqa: shape mismatch")
+    if tuple(lse.shape) != (B, H, Nq) or lse.dtype != torch.float32:
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_fwd_gqa: lse must be fp32 [B, H, Nq]")
+    if not (q.dtype == k.dtype == v.dtype == o.dtype):
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_fwd_gqa: dtype mismatch")
+    st = load_library().mea_attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Nq, Nk, D,
+                                          float(scale), _dtype_code(q), _stream_handle(stream))
+    _check(st, "mea_attn_fwd_gqa")
+
+
+def mea_attn_bwd_gqa_workspace_size(B: int, H: int, H_kv: int, Nq: int, Nk: int, D: int,
+                                    dtype=torch.bfloat16) -> int:
+    out = ctypes.c_size_t(0)
+    code = MEA_DTYPE_BF16 if dtype == torch.bfloat16 else MEA_DTYPE_F32
+    st = load_library().mea_attn_bwd_gqa_workspace_size(B, H, H_kv, Nq, Nk, D, code, ctypes.byref(out))
+    _check(st, "mea_attn_bwd_gqa_workspace_size")
+    return int(out.value)
+
+
+def mea_attn_bwd_gqa(q, k, v, o, lse, do, dq, dk, dv, scale: float, workspace, stream=None) -> None:
+    """C ``mea_attn_bwd_gqa``: dq [B,H,Nq,D]; dk, dv [B,H_kv,Nk,D] summed over each group."""
+    B, H, Hkv, Nq, Nk, D = _gqa_shapes(q, k, "mea_attn_bwd_gqa")
+    for name, t, shape in (("o", o, q.shape), ("do", do, q.shape), ("dq", dq, q.shape), ("v", v, k.shape),
+                           ("dk", dk, k.shape), ("dv", dv, k.shape)):
+        if tuple(t.shape) != tuple(shape) or t.dtype != q.dtype:
+            raise MeaError(MEA_ERR_INVALID_ARG, f"mea_attn_bwd_gqa: {name} shape/dtype mismatch")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load_library().mea_attn_bwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq),
+                                          _ptr(dk), _ptr(dv), B, H, Hkv, Nq, Nk, D, float(scale), _dtype_code(q),
+                                          _ptr(workspace), ws_bytes, _stream_handle(stream))
+    _check(st, "mea_attn_bwd_gqa")
+
+
 def mea_selftest_bounded_wait(gave_up, stream=None) -> None:
     """C ``mea_selftest_bounded_wait``: a kernel whose bounded wait must expire (about 1 s)."""
     if gave_up.dtype != torch.int32 or not gave_up.is_cuda or gave_up.numel() < 1:
@@ -220,7 +276,10 @@ def attention_forward(q, k, v, scale: float | None = None, stream=None):
         scale = 1.0 / math.sqrt(q.shape[-1])
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
-    mea_attn_fwd(q, k, v, o, lse, scale, stream)
+    if k.dim() == 4 and q.dim() == 4 and k.shape[1] != q.shape[1]:
+        mea_attn_fwd_gqa(q, k, v, o, lse, scale, stream)
+    else:
+        mea_attn_fwd(q, k, v, o, lse, scale, stream)
     return o, lse
 
 
@@ -229,12 +288,15 @@ def attention_backward(q, k, v, o, lse, do, scale: float | None = None, workspac
     if scale is None:
         scale = 1.0 / math.sqrt(q.shape[-1])
     B, H, Nq, D = q.shape
-    Nk = k.shape[2]
+    Hkv, Nk = k.shape[1], k.shape[2]
     if workspace is None:
-        workspace = torch.empty(mea_attn_bwd_workspace_size(B, H, Nq, Nk, D, q.dtype), dtype=torch.uint8,
+        workspace = torch.empty(mea_attn_bwd_gqa_workspace_size(B, H, Hkv, Nq, Nk, D, q.dtype), dtype=torch.uint8,
                                 device=q.device)
     dq = torch.empty_like(q)
     dk = torch.empty_like(k)
     dv = torch.empty_like(v)
-    mea_attn_bwd(q, k, v, o, lse, do, dq, dk, dv, scale, workspace, stream)
+    if Hkv != H:
+        mea_attn_bwd_gqa(q, k, v, o, lse, do, dq, dk, dv, scale, workspace, stream)
+    else:
+        mea_attn_bwd(q, k, v, o, lse, do, dq, dk, dv, scale, workspace, stream)
     return dq, dk, dv

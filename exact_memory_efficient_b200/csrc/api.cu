@@ -317,6 +317,54 @@ mea_status_t mea_attn_bwd(const void* q, const void* k, const void* v, const voi
 }
 
 // ---------------------------------------------------------------------------
+// Shared key/value heads.  The G = H / H_kv query heads of one group are
+// consecutive in [B, H, Nq, D], so they are one contiguous [G*Nq, D] block:
+// the group is a single "head" of G*Nq query rows over its key/value head,
+// and the kernels above run unchanged over B*H_kv such heads.  lse, the dQ
+// accumulator and the row term D_i follow the same [B*H_kv, G*Nq] view.
+}  // extern "C"
+
+namespace {
+mea_status_t gqa_rows(int H, int H_kv, int Nq, int* rows) {
+    if (H < 0 || H_kv < 1 || Nq < 0 || H % H_kv != 0)
+        return fail(MEA_ERR_INVALID_ARG, "gqa", "H must be a multiple of H_kv >= 1");
+    const long long r = (long long)(H / H_kv) * Nq;
+    if (r > 0x7fffffffLL) return fail(MEA_ERR_UNSUPPORTED, "gqa", "(H / H_kv) * Nq exceeds 2^31-1");
+    *rows = (int)r;
+    return MEA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+mea_status_t mea_attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                              int H_kv, int Nq, int Nk, int D, float scale, mea_dtype_t dtype, void* stream) {
+    int rows = 0;
+    mea_status_t st = gqa_rows(H, H_kv, Nq, &rows);
+    if (st != MEA_OK) return st;
+    return mea_attn_fwd(q, k, v, o, lse, B, H_kv, rows, Nk, D, scale, dtype, stream);
+}
+
+mea_status_t mea_attn_bwd_gqa_workspace_size(int B, int H, int H_kv, int Nq, int Nk, int D, mea_dtype_t dtype,
+                                             size_t* bytes) {
+    int rows = 0;
+    mea_status_t st = gqa_rows(H, H_kv, Nq, &rows);
+    if (st != MEA_OK) return st;
+    return mea_attn_bwd_workspace_size(B, H_kv, rows, Nk, D, dtype, bytes);
+}
+
+mea_status_t mea_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                              const void* dO, void* dq, void* dk, void* dv, int B, int H, int H_kv, int Nq, int Nk,
+                              int D, float scale, mea_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+    int rows = 0;
+    mea_status_t st = gqa_rows(H, H_kv, Nq, &rows);
+    if (st != MEA_OK) return st;
+    return mea_attn_bwd_phase(MEA_BWD_ALL, q, k, v, o, lse, dO, dq, dk, dv, B, H_kv, rows, Nk, D, scale, dtype,
+                              workspace, workspace_bytes, stream);
+}
+
+// ---------------------------------------------------------------------------
 // Backward without any allocation, for callers that cannot allocate device
 // memory (see mea_attn_bwd_noalloc in mea_attn.h).  The scratch lives in one
 // file-scope device array that every device loading this library keeps until

@@ -150,6 +150,45 @@ mea_status_t mea_attn_bwd_phase(mea_bwd_phase_t phase,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Shared key/value heads: grouped-query (1 < H_kv < H) and multi-query
+ * (H_kv == 1) attention.
+ *
+ * Source: "当注意力成为瓶颈从on困境到线性复杂度的技术突围" (section
+ * 推理优化：减少KV Cache): the query heads are split into groups and each
+ * group shares one key/value head.  Reading adopted: the groups are
+ * consecutive, so query head h uses key/value head h / (H / H_kv).  The
+ * gradient of a shared key/value head is the sum over the query heads of its
+ * group.
+ *
+ * Layout: q, o, dO, dq [B, H, Nq, D]; k, v, dk, dv [B, H_kv, Nk, D];
+ * lse [B, H, Nq] fp32.  Because the G = H / H_kv query heads of a group are
+ * consecutive, they form one contiguous [G*Nq, D] block of q, so each call
+ * runs the kernels of mea_attn_fwd / mea_attn_bwd over B*H_kv heads of G*Nq
+ * query rows: every key/value tile is loaded once per group, and dk, dv sum
+ * over the group inside one accumulator (no atomics, deterministic).
+ *
+ * Arguments, ownership, alignment, supported dtypes and head dims, and errors
+ * are those of the entry point without the suffix, plus: H_kv < 1 or H not a
+ * multiple of H_kv returns MEA_ERR_INVALID_ARG; G*Nq above 2^31-1 returns
+ * MEA_ERR_UNSUPPORTED.  H == 0 is a no-op for the forward; the backward then
+ * writes zeros to dk, dv.  H_kv == H is exactly mea_attn_fwd / mea_attn_bwd.
+ */
+mea_status_t mea_attn_fwd_gqa(const void* q, const void* k, const void* v,
+                              void* o, float* lse,
+                              int B, int H, int H_kv, int Nq, int Nk, int D, float scale,
+                              mea_dtype_t dtype, void* stream);
+
+mea_status_t mea_attn_bwd_gqa_workspace_size(int B, int H, int H_kv, int Nq, int Nk, int D,
+                                             mea_dtype_t dtype, size_t* bytes);
+
+mea_status_t mea_attn_bwd_gqa(const void* q, const void* k, const void* v,
+                              const void* o, const float* lse, const void* dO,
+                              void* dq, void* dk, void* dv,
+                              int B, int H, int H_kv, int Nq, int Nk, int D, float scale,
+                              mea_dtype_t dtype,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Backward pass that allocates nothing and takes no workspace.  The paper has
  * no counterpart: this is a deployment convenience of this library.
  *

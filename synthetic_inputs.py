@@ -6,7 +6,9 @@ and the fp64 oracle consume exactly the tensors produced here (the oracle takes
 their exact fp64 upcast), so neither side generates data for the other.
 
 Recipe (all workloads): ``torch.Generator('cpu').manual_seed(seed)``, then
-``torch.randn`` in fp32 in the order Q, K, V, dO; Q and K are multiplied by
+``torch.randn`` in fp32 in the order Q, K, V, dO (K and V with the workload's
+key/value head count, which equals the query head count unless the workload
+shares key/value heads); Q and K are multiplied by
 ``qk_mult`` in fp32 (the single-query workload uses 40 so that logits reach
 the +-1e3 range that a max-free exponential cannot represent); finally the
 tensors are cast (round-to-nearest-even) to the workload dtype.  Layout is
@@ -34,6 +36,11 @@ class Workload:
     backward: bool
     qk_mult: float = 1.0
     note: str = ""
+    Hkv: int | None = None  # key/value heads (None: one per query head)
+
+    @property
+    def H_kv(self) -> int:
+        return self.H if self.Hkv is None else self.Hkv
 
     @property
     def scale(self) -> float:
@@ -44,6 +51,7 @@ class Workload:
         return torch.float32 if self.dtype == "f32" else torch.bfloat16
 
     def fwd_flops(self) -> float:
+        # shared key/value heads change the bytes read, not the flops
         # 4 * B * H * Nq * Nk * D: two GEMMs of 2*Nq*Nk*D each per head.
         return 4.0 * self.B * self.H * self.Nq * self.Nk * self.D
 
@@ -64,6 +72,13 @@ WORKLOADS = {
 }
 WORKLOADS["decode_16384_bf16"] = Workload("decode_16384_bf16", 1, 8, 1, 16384, 128, "bf16", False,
                                           note="decode-shaped bf16 forward: one query row over 16384 keys, 8 heads")
+# Shared key/value heads, with the grouping the survey page gives as its example
+# (32 query heads in 8 groups of 4).
+WORKLOADS["gqa_32x8_4096_bf16"] = Workload("gqa_32x8_4096_bf16", 1, 32, 4096, 4096, 128, "bf16", True, Hkv=8,
+                                           note="grouped-query attention: 32 query heads, 8 key/value heads")
+WORKLOADS["decode_gqa_32x8_16384_bf16"] = Workload(
+    "decode_gqa_32x8_16384_bf16", 1, 32, 1, 16384, 128, "bf16", False, Hkv=8,
+    note="decode-shaped grouped-query forward: one query row per head, 32 query heads over 8 key/value heads")
 for _n in (256, 1024, 4096, 16384):
     WORKLOADS[f"long_{_n}_bf16"] = Workload(f"long_{_n}_bf16", 1, 16, _n, _n, 128, "bf16", True,
                                              note=f"long-sequence sweep B1 H16 N{_n} D128")
@@ -74,8 +89,8 @@ def make_workload(name: str) -> Workload:
 
 
 def custom(B: int, H: int, Nq: int, Nk: int, D: int, dtype: str, backward: bool = True,
-           qk_mult: float = 1.0, name: str = "custom") -> Workload:
-    return Workload(name, B, H, Nq, Nk, D, dtype, backward, qk_mult)
+           qk_mult: float = 1.0, name: str = "custom", Hkv: int | None = None) -> Workload:
+    return Workload(name, B, H, Nq, Nk, D, dtype, backward, qk_mult, Hkv=Hkv)
 
 
 def make_inputs(w: Workload, seed: int, with_grad_output: bool | None = None):
@@ -88,8 +103,8 @@ def make_inputs(w: Workload, seed: int, with_grad_output: bool | None = None):
     g = torch.Generator(device="cpu")
     g.manual_seed(int(seed))
     q = torch.randn((w.B, w.H, w.Nq, w.D), generator=g, dtype=torch.float32)
-    k = torch.randn((w.B, w.H, w.Nk, w.D), generator=g, dtype=torch.float32)
-    v = torch.randn((w.B, w.H, w.Nk, w.D), generator=g, dtype=torch.float32)
+    k = torch.randn((w.B, w.H_kv, w.Nk, w.D), generator=g, dtype=torch.float32)
+    v = torch.randn((w.B, w.H_kv, w.Nk, w.D), generator=g, dtype=torch.float32)
     want_do = w.backward if with_grad_output is None else with_grad_output
     do = torch.randn((w.B, w.H, w.Nq, w.D), generator=g, dtype=torch.float32) if want_do else None
     if w.qk_mult != 1.0:

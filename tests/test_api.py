@@ -133,3 +133,31 @@ def test_python_binding_rejects_bad_tensors(lib):
         m.mea_attn_fwd(q, q, q, q, torch.zeros(1, 1, 4), 0.125)  # CPU tensors are rejected
     with pytest.raises(m.MeaError):
         m.mea_attn_fwd(q[0], q, q, q, torch.zeros(1, 1, 4), 0.125)
+
+
+def test_gqa_argument_validation(lib):
+    def fwd_gqa(H=4, Hkv=2, Nq=16, q=A, B=1):
+        return lib.mea_attn_fwd_gqa(q, A, A, A, A, B, H, Hkv, Nq, 16, 64, ctypes.c_float(0.125), BF16, None)
+
+    def bwd_gqa(H=4, Hkv=2, Nq=16, ws=A, ws_bytes=1 << 30, D=64):
+        return lib.mea_attn_bwd_gqa(*([A] * 9), 1, H, Hkv, Nq, 16, D, ctypes.c_float(0.125), BF16, ws, ws_bytes,
+                                    None)
+
+    assert fwd_gqa(Hkv=3) == 1            # H not a multiple of H_kv
+    assert fwd_gqa(Hkv=0) == 1
+    assert fwd_gqa(Hkv=-2) == 1
+    assert fwd_gqa(H=1 << 20, Hkv=1, Nq=1 << 12) == 2   # group rows exceed 2^31-1
+    assert fwd_gqa(q=None) == 1
+    assert fwd_gqa(q=A + 8) == 3
+    assert fwd_gqa(Nq=0) == 0             # no rows: no-op
+    assert fwd_gqa(H=0, Hkv=1) == 0
+    assert bwd_gqa(Hkv=3) == 1
+    assert bwd_gqa(D=96) == 2
+    assert bwd_gqa(ws=None) == 4
+    out = ctypes.c_size_t(0)
+    assert lib.mea_attn_bwd_gqa_workspace_size(1, 4, 3, 16, 16, 64, BF16, ctypes.byref(out)) == 1
+    # the workspace follows the query heads: the same bytes as the per-head backward with H heads
+    ref = ctypes.c_size_t(0)
+    assert lib.mea_attn_bwd_gqa_workspace_size(2, 32, 8, 100, 300, 128, BF16, ctypes.byref(out)) == 0
+    assert lib.mea_attn_bwd_workspace_size(2, 32, 100, 300, 128, BF16, ctypes.byref(ref)) == 0
+    assert out.value == ref.value
