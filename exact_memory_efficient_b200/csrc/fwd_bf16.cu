@@ -117,6 +117,9 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     asm("mov.u32 %0, %%cluster_nctarank;" : "=r"(nranks));
     asm("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
     const int m0 = (blockIdx.x / nranks) * (2 * kTileM);
+    // A CTA whose rows all fall in its first query tile (decode-shaped calls,
+    // the last tile pair of a ragged Nq) issues no work for the second tile.
+    const bool two = (m0 + kTileM) < Nq;
     const int c_begin = (nranks > 1) ? (int)rank * chunk_len : 0;
     const int c_end = (nranks > 1) ? min(Nk, c_begin + chunk_len) : Nk;
     const int n_kv = (c_end > c_begin) ? (c_end - c_begin + kTileN - 1) / kTileN : 0;
@@ -152,8 +155,9 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
-            mbar_arrive_expect_tx(&bars->q_full, 2 * Cfg::kQBytes);
-            for (int t = 0; t < 2; ++t)
+            const int n_qt = two ? 2 : 1;
+            mbar_arrive_expect_tx(&bars->q_full, n_qt * Cfg::kQBytes);
+            for (int t = 0; t < n_qt; ++t)
                 for (int b = 0; b < D / 64; ++b)
                     tma_load_3d(sQ + t * Cfg::kQBytes + b * Cfg::kBoxBytes, &tm_q, &bars->q_full,
                                 b * 64, m0 + t * kTileM, bh);
@@ -237,8 +241,10 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc_fence_after();
                 issue_s(tS0, q_lo0, k_off);
                 mma_commit(&bars->s_full[0]);
-                issue_s(tS1, q_lo1, k_off);
-                mma_commit(&bars->s_full[1]);
+                if (two) {
+                    issue_s(tS1, q_lo1, k_off);
+                    mma_commit(&bars->s_full[1]);
+                }
                 mma_commit(&bars->empty[k_stage]);
             }
             for (int j = 0; ok && j < n_kv; ++j) {
@@ -258,13 +264,17 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     mma_commit(&bars->s_full[0]);
                 }
                 // tile 1: O_1 += P_1 V_j, then S_1 = Q_1 K_{j+1}^T
-                if (!(ok = mbar_wait(&bars->p_ready[1], j & 1, abort_flag))) break;
-                tc_fence_after();
-                issue_pv(tO1, tS1, v_off, acc0);
+                if (two) {
+                    if (!(ok = mbar_wait(&bars->p_ready[1], j & 1, abort_flag))) break;
+                    tc_fence_after();
+                    issue_pv(tO1, tS1, v_off, acc0);
+                }
                 mma_commit(&bars->empty[v_stage]);
                 if (more) {
-                    issue_s(tS1, q_lo1, k_off);
-                    mma_commit(&bars->s_full[1]);
+                    if (two) {
+                        issue_s(tS1, q_lo1, k_off);
+                        mma_commit(&bars->s_full[1]);
+                    }
                     mma_commit(&bars->empty[k_stage]);
                 }
             }
@@ -281,6 +291,18 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const unsigned lane_off = (sub * 32u) << 16;
         const unsigned tS = tmem + lane_off + (t ? 128u : 0u);
         const unsigned tO = tmem + lane_off + (t ? 384u : 256u);
+        // Rows at or past Nq are never stored and a row of O depends only on
+        // the same row of P, so a warp whose 32 rows all lie past Nq only keeps
+        // the handshake (its P lanes hold whatever S left there), and the warps
+        // of an unused second tile take no part at all.
+        if ((m0 + t * kTileM + (int)sub * 32) >= Nq) {
+            if (t == 0 || two) {
+                for (int j = 0; j < n_kv; ++j) {
+                    if (!mbar_wait(&bars->s_full[t], j & 1, abort_flag)) break;
+                    mbar_arrive(&bars->p_ready[t]);
+                }
+            }
+        } else {
         const float c_log2 = scale * kLog2e;
         float m_ref = -INFINITY;  // reference maximum, base-2 units of scale*s
         float l = 0.f;
@@ -404,6 +426,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 ml[1] = (n_kv > 0) ? l : 0.f;
             }
         }
+        }  // rows of this warp below Nq
     }
 
     if (nranks > 1) {
