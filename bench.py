@@ -52,24 +52,33 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_sha() -> str:
+def source_sha(names=None) -> str:
+    """Hash of the CUDA sources (all of them, or the named files)."""
     h = hashlib.sha256()
     for name in sorted(os.listdir(CSRC)):
-        if name.endswith((".cu", ".cuh", ".h")):
+        if name.endswith((".cu", ".cuh", ".h")) and (names is None or name in names):
             with open(os.path.join(CSRC, name), "rb") as f:
                 h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
+# the files whose text decides each timed kernel's code
+KERNEL_SOURCES = {
+    "bwd_main_kernel": ("bwd_bf16.cu", "ptx.cuh", "kernels.h"),
+    "fwd_bf16_kernel": ("fwd_bf16.cu", "ptx.cuh", "kernels.h"),
+}
+
+
 def ncu_traffic(kernel: str):
-    """DRAM bytes per launch from a committed ncu summary, if it matches the current sources."""
+    """DRAM bytes per launch from a committed ncu summary, if the kernel's sources are unchanged since."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel)
-    if not e or e.get("src_sha") != source_sha():
+    base = kernel.split("<")[0]
+    if not e or base not in KERNEL_SOURCES or e.get("src_sha") != source_sha(KERNEL_SOURCES[base]):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -85,6 +94,24 @@ class ClockSampler:
         self.dev = device_index
         self.proc = None
         self.path = None
+        self.fine = []
+        self._stop = False
+        self._thread = None
+        self._nvml = None
+
+    def _nvml_loop(self):
+        # Finer record through NVML (read-only queries), every 5 ms: SM clock
+        # and the event-reason mask (0x4 software power cap, 0x8 hardware
+        # slowdown, 0x20 software thermal, 0x40 hardware thermal).
+        import pynvml
+        h = self._nvml
+        while not self._stop:
+            try:
+                self.fine.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                  int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))))
+            except Exception:  # noqa: BLE001
+                return
+            time.sleep(0.005)
 
     def start(self):
         fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
@@ -96,8 +123,34 @@ class ClockSampler:
         except (FileNotFoundError, OSError):
             self.proc = None
         time.sleep(0.3)
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml.nvmlDeviceGetHandleByIndex(self.dev)
+        except Exception:  # noqa: BLE001 - NVML missing: keep the nvidia-smi record only
+            return
+        import threading
+        self._thread = threading.Thread(target=self._nvml_loop, daemon=True)
+        self._thread.start()
+
+    def fine_summary(self):
+        self._stop = True
+        if self._thread is not None:
+            self._thread.join(timeout=2)
+        if not self.fine:
+            return None
+        sm = [c for c, _ in self.fine]
+        return {"samples": len(sm), "period_ms": 5, "sm_mhz_median": statistics.median(sm), "sm_mhz_min": min(sm),
+                "sw_power_cap_frac": round(sum(1 for _, r in self.fine if r & 0x4) / len(sm), 3),
+                "hw_or_thermal_slowdown": any(r & (0x8 | 0x20 | 0x40) for _, r in self.fine)}
 
     def stop(self):
+        fine = self.fine_summary()
+        out = self._stop_smi()
+        out["nvml_5ms"] = fine
+        return out
+
+    def _stop_smi(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         time.sleep(0.2)
@@ -325,29 +378,63 @@ def run_ours(args):
                                                "finalize": round(statistics.mean(fin_ms), 4)}}
     if rank == 0 and not args.no_extras:
         # HBM-bound decode-shaped forwards, timed one launch at a time with L2
-        # flushed in between (their K/V would otherwise stay L2-resident)
-        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-        for wname in ("single_query_f32", "decode_16384_bf16"):
+        # flushed in between (their K/V would otherwise stay L2-resident).  The
+        # flush reads a 256 MB buffer, so it leaves no dirty lines for the timed
+        # kernel to write back; a sleep kernel queued first lets the host
+        # enqueue every launch before the GPU reaches them, so the events time
+        # the kernels and not the host's launch path.
+        flush = torch.zeros(64 << 20, dtype=torch.float32, device=dev)
+        for wname in ("single_query_f32", "decode_16384_bf16", "decode_gqa_32x8_16384_bf16"):
             wd = make_workload(wname)
             qd, kd, vd, _ = (x.to(dev) if x is not None else None for x in make_inputs(wd, 0))
             od, ld = m.attention_forward(qd, kd, vd, wd.scale)
             for _ in range(3):
-                m.mea_attn_fwd(qd, kd, vd, od, ld, wd.scale)
+                m.mea_attn_fwd_gqa(qd, kd, vd, od, ld, wd.scale)
             reps = 20
             evs_d = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+            torch.cuda.synchronize()
+            torch.cuda._sleep(40_000_000)
             for e0, e1 in evs_d:
-                flush.zero_()
+                flush.sum()
                 e0.record(stream)
-                m.mea_attn_fwd(qd, kd, vd, od, ld, wd.scale)
+                m.mea_attn_fwd_gqa(qd, kd, vd, od, ld, wd.scale)
                 e1.record(stream)
             torch.cuda.synchronize()
             us = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs_d) * 1e3
             byts = sum(x.numel() * x.element_size() for x in (qd, kd, vd, od, ld))
             rows[f"{wname}_fwd"] = {"us": round(us, 2), "GB/s": round(byts / (us * 1e-6) / 1e9, 1),
                                     "frac_of_hbm": round(byts / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 3),
-                                    "bytes": byts, "note": "median of 20 launches, L2 flushed before each"}
+                                    "bytes": byts, "H_kv": wd.H_kv,
+                                    "note": "median of 20 launches, L2 flushed (256 MB read) before each"}
             del qd, kd, vd, od, ld
         del flush
+        # grouped-query forward + backward (32 query heads over 8 key/value heads)
+        wg = make_workload("gqa_32x8_4096_bf16")
+        qg, kg, vg, dog = (x.to(dev) for x in make_inputs(wg, 0))
+        og, lg = m.attention_forward(qg, kg, vg, wg.scale)
+        wsg = torch.empty(m.mea_attn_bwd_gqa_workspace_size(wg.B, wg.H, wg.H_kv, wg.Nq, wg.Nk, wg.D),
+                          dtype=torch.uint8, device=dev)
+        grads = [torch.empty_like(x) for x in (qg, kg, vg)]
+        for _ in range(3):
+            m.mea_attn_fwd_gqa(qg, kg, vg, og, lg, wg.scale)
+            m.mea_attn_bwd_gqa(qg, kg, vg, og, lg, dog, *grads, wg.scale, wsg)
+        reps = 10
+        ev_g = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+        for e in ev_g:
+            e[0].record(stream)
+            m.mea_attn_fwd_gqa(qg, kg, vg, og, lg, wg.scale)
+            e[1].record(stream)
+            m.mea_attn_bwd_gqa(qg, kg, vg, og, lg, dog, *grads, wg.scale, wsg)
+            e[2].record(stream)
+        torch.cuda.synchronize()
+        f_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev_g)
+        b_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev_g)
+        rows[f"{wg.name}_fwd"] = {"ms": round(f_ms, 4), "TFLOP/s": round(wg.fwd_flops() / (f_ms * 1e-3) / 1e12, 1),
+                                  "frac_of_peak": round(wg.fwd_flops() / (f_ms * 1e-3) / 1e12 / peak, 3)}
+        rows[f"{wg.name}_bwd"] = {"ms": round(b_ms, 4), "TFLOP/s": round(wg.bwd_flops() / (b_ms * 1e-3) / 1e12, 1),
+                                  "frac_of_peak": round(wg.bwd_flops() / (b_ms * 1e-3) / 1e12 / peak, 3),
+                                  "note": f"mean of {reps}; inputs ({wg.H}+2x{wg.H_kv} heads) fit in L2"}
+        del qg, kg, vg, dog, og, lg, wsg, grads
 
     # ---- extra memory versus a materialised-scores attention (arithmetic)
     naive_scores = w.B * w.H * w.Nq * w.Nk * 4
