@@ -240,8 +240,12 @@ mea_status_t mea_attn_bwd_workspace_size(int B, int H, int Nq, int Nk, int D, me
     if (bytes == nullptr) return MEA_ERR_INVALID_ARG;
     mea_status_t st = common_checks(B, H, Nq, Nk, D, 1.0f, dtype);
     if (st != MEA_OK) return st;
-    if (dtype != MEA_DTYPE_BF16) return MEA_ERR_UNSUPPORTED;
     const size_t rows = (size_t)B * H * Nq;
+    if (dtype == MEA_DTYPE_F32) {
+        // fp32: the row term only (dQ is summed per row in registers)
+        *bytes = round_up(rows * sizeof(float), 256);
+        return MEA_OK;
+    }
     *bytes = round_up(rows * D * sizeof(float), 256) + round_up(rows * sizeof(float), 256);
     return MEA_OK;
 }
@@ -260,15 +264,15 @@ mea_status_t mea_attn_bwd_phase(mea_bwd_phase_t phase, const void* q, const void
     }
     mea_status_t st = common_checks(B, H, Nq, Nk, D, scale, dtype);
     if (st != MEA_OK) return st;
-    if (dtype != MEA_DTYPE_BF16) return MEA_ERR_UNSUPPORTED;
     const int BH = B * H;
     if (BH == 0) return MEA_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t esize = dtype == MEA_DTYPE_F32 ? 4 : 2;
     if (Nq == 0) {
         if (Nk == 0 || !(phases & mea::kBwdPhaseMain)) return MEA_OK;
         if (!dk || !dv) return MEA_ERR_INVALID_ARG;
         if (!aligned16(dk) || !aligned16(dv)) return MEA_ERR_MISALIGNED;
-        const size_t n = (size_t)BH * Nk * D * 2;
+        const size_t n = (size_t)BH * Nk * D * esize;
         cudaError_t e = cudaMemsetAsync(dk, 0, n, s);
         if (e != cudaSuccess) return fail_cuda("cudaMemsetAsync", e);
         return cuda_status(cudaMemsetAsync(dv, 0, n, s), "cudaMemsetAsync");
@@ -285,6 +289,35 @@ mea_status_t mea_attn_bwd_phase(mea_bwd_phase_t phase, const void* q, const void
     DeviceInfo* dev = nullptr;
     if ((st = device_info(&dev)) != MEA_OK) return st;
     if (BH > 65535) return MEA_ERR_UNSUPPORTED;
+
+    if (dtype == MEA_DTYPE_F32) {
+        mea::F32BwdArgs f;
+        f.q = static_cast<const float*>(q);
+        f.k = static_cast<const float*>(k);
+        f.v = static_cast<const float*>(v);
+        f.o = static_cast<const float*>(o);
+        f.dO = static_cast<const float*>(dO);
+        f.lse = lse;
+        f.dq = static_cast<float*>(dq);
+        f.dk = static_cast<float*>(dk);
+        f.dv = static_cast<float*>(dv);
+        f.delta = static_cast<float*>(workspace);
+        f.BH = BH;
+        f.Nq = Nq;
+        f.Nk = Nk;
+        f.D = D;
+        f.scale = scale;
+        // Rows per CTA of 8 warps: fewer rows (more warps sharing one row's
+        // loop) while the grid would leave SMs idle.
+        auto rows_per_cta = [&](int rows) {
+            int r = 8;
+            while (r > 1 && (long long)BH * ((rows + r - 1) / r) < 2LL * dev->sm_count) r /= 2;
+            return r;
+        };
+        f.q_rows_per_cta = rows_per_cta(Nq);
+        f.k_rows_per_cta = rows_per_cta(Nk);
+        return cuda_status(mea::launch_bwd_f32(f, s, phases), "bwd_f32 launch");
+    }
 
     mea::Bf16BwdArgs a;
     if ((st = make_map(&a.tm_q, q, BH, Nq, D)) != MEA_OK) return st;

@@ -25,6 +25,25 @@ struct F32FwdArgs {
 };
 cudaError_t launch_fwd_f32(const F32FwdArgs& a, cudaStream_t stream);
 
+// fp32 SIMT backward (bwd_f32.cu).  Row term D_i in `delta` (workspace).
+struct F32BwdArgs {
+    const float* q;
+    const float* k;
+    const float* v;
+    const float* o;
+    const float* dO;
+    const float* lse;
+    float* dq;
+    float* dk;
+    float* dv;
+    float* delta;       // [BH, Nq]
+    int BH, Nq, Nk, D;
+    float scale;
+    int q_rows_per_cta;  // dQ kernel: query rows per CTA of 8 warps (1, 2, 4 or 8)
+    int k_rows_per_cta;  // dK/dV kernel: key rows per CTA of 8 warps (1, 2, 4 or 8)
+};
+cudaError_t launch_bwd_f32(const F32BwdArgs& a, cudaStream_t stream, unsigned phases);
+
 // bf16 tcgen05 forward (fwd_bf16.cu).  Tensor maps are 3-D {D, N, B*H} bf16,
 // 128-byte swizzle, box {64, 128, 1}.
 struct Bf16FwdArgs {

@@ -38,7 +38,8 @@
  * Supported set
  *  - MEA_DTYPE_BF16: forward and backward, D in {64, 128}; inputs/outputs bf16,
  *    accumulation fp32 (tcgen05 tensor cores).
- *  - MEA_DTYPE_F32: forward only, D in {32, 64, 96, 128}; fp32 throughout.
+ *  - MEA_DTYPE_F32: forward and backward, D in {32, 64, 96, 128}; fp32
+ *    throughout (SIMT kernels, no tensor cores).
  *  - Any Nq >= 0 and Nk >= 1; partial tiles are masked.  No mask, no dropout.
  *  - B*H <= 2^31-1 and B*H*max(Nq,Nk)*D < 2^40 elements.
  */
@@ -88,10 +89,10 @@ mea_status_t mea_attn_fwd(const void* q, const void* k, const void* v,
 
 /*
  * Bytes of device workspace mea_attn_bwd needs for these sizes (written to
- * *bytes): an fp32 dQ accumulator [B,H,Nq,D] and the fp32 row term
- * D_i = sum_d dO_id O_id [B,H,Nq], each 256-byte aligned.  O(N*D), never
- * O(N^2).  Errors: MEA_ERR_INVALID_ARG (null `bytes`, negative size),
- * MEA_ERR_UNSUPPORTED (dtype/D not supported for backward).
+ * *bytes).  bf16: an fp32 dQ accumulator [B,H,Nq,D] and the fp32 row term
+ * D_i = sum_d dO_id O_id [B,H,Nq], each 256-byte aligned.  fp32: the row term
+ * only.  O(N*D), never O(N^2).  Errors: MEA_ERR_INVALID_ARG (null `bytes`,
+ * negative size), MEA_ERR_UNSUPPORTED (dtype/D not supported).
  */
 mea_status_t mea_attn_bwd_workspace_size(int B, int H, int Nq, int Nk, int D,
                                          mea_dtype_t dtype, size_t* bytes);
@@ -109,10 +110,11 @@ mea_status_t mea_attn_bwd_workspace_size(int B, int H, int Nq, int Nk, int D,
  * q,k,v,o,dO inputs (dtype); lse input fp32 [B,H,Nq] from mea_attn_fwd;
  * dq,dk,dv outputs (dtype).  workspace: device memory of at least
  * mea_attn_bwd_workspace_size() bytes, owned by the caller, contents on entry
- * ignored, clobbered on exit.  dq is accumulated in fp32 with atomic adds, so it
- * is not bitwise deterministic run to run (dk, dv are).
- * Nq == 0 writes zeros to dk, dv.  Errors as for mea_attn_fwd plus
- * MEA_ERR_WORKSPACE; MEA_DTYPE_F32 returns MEA_ERR_UNSUPPORTED.
+ * ignored, clobbered on exit.  bf16: dq is accumulated in fp32 by reduce-adds
+ * from many CTAs, so it is not bitwise deterministic run to run (dk, dv are).
+ * fp32: dq, dk, dv are each summed by one CTA in a fixed order (bitwise
+ * deterministic).  Nq == 0 writes zeros to dk, dv.  Errors as for
+ * mea_attn_fwd plus MEA_ERR_WORKSPACE.
  */
 mea_status_t mea_attn_bwd(const void* q, const void* k, const void* v,
                           const void* o, const float* lse, const void* dO,
@@ -132,6 +134,8 @@ mea_status_t mea_attn_bwd(const void* q, const void* k, const void* v,
  *   MEA_BWD_MAIN        recomputes P from lse per key tile; writes dk, dv and
  *                       adds dS K into the dQ accumulator.  (reads q, k, v, dO, lse)
  *   MEA_BWD_FINALIZE    dq = bf16(scale * dQ accumulator). (writes dq)
+ * For MEA_DTYPE_F32 the main phase writes dq, dk and dv directly and the
+ * preprocess phase only computes D_i; the finalize phase does nothing.
  * Errors as for mea_attn_bwd; an unknown phase returns MEA_ERR_INVALID_ARG.
  */
 typedef enum {
@@ -202,7 +206,8 @@ mea_status_t mea_attn_bwd_gqa(const void* q, const void* k, const void* v,
  * until the process exits.
  *
  * Arguments, layout, results and errors are those of mea_attn_bwd without the
- * workspace pair.  Sizes whose workspace (mea_attn_bwd_workspace_size) exceeds
+ * workspace pair, for MEA_DTYPE_BF16 only (MEA_DTYPE_F32 returns
+ * MEA_ERR_UNSUPPORTED).  Sizes whose workspace (mea_attn_bwd_workspace_size) exceeds
  * MEA_NOALLOC_SCRATCH_BYTES are rejected with MEA_ERR_WORKSPACE and a message
  * in mea_last_error_message().  The first call on each device resolves the
  * array's device address (cudaGetSymbolAddress) with that device current; make

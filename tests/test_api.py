@@ -87,7 +87,8 @@ def test_forward_empty_is_noop(lib):
 
 
 def test_backward_argument_validation(lib):
-    assert bwd(lib, dtype=F32) == 2
+    assert bwd(lib, dtype=F32, D=48) == 2   # fp32 needs D % 32 == 0 and D <= 128
+    assert bwd(lib, dtype=F32, D=160) == 2
     assert bwd(lib, D=96) == 2
     assert bwd(lib, Nk=0) == 1
     assert bwd(lib, Nq=-3) == 1
@@ -116,7 +117,12 @@ def test_workspace_size(lib):
     assert lib.mea_attn_bwd_workspace_size(2, 3, 5, 7, 64, BF16, ctypes.byref(out)) == 0
     r = 2 * 3 * 5
     assert out.value == ((r * 64 * 4 + 255) // 256) * 256 + ((r * 4 + 255) // 256) * 256
-    assert lib.mea_attn_bwd_workspace_size(1, 1, 4, 4, 64, F32, ctypes.byref(out)) == 2
+    # fp32: the row term only
+    assert lib.mea_attn_bwd_workspace_size(1, 1, 4, 4, 64, F32, ctypes.byref(out)) == 0
+    assert out.value == 256
+    assert lib.mea_attn_bwd_workspace_size(2, 3, 1000, 4, 96, F32, ctypes.byref(out)) == 0
+    assert out.value == ((2 * 3 * 1000 * 4 + 255) // 256) * 256
+    assert lib.mea_attn_bwd_workspace_size(1, 1, 4, 4, 48, F32, ctypes.byref(out)) == 2
     assert lib.mea_attn_bwd_workspace_size(1, 1, 4, 4, 64, BF16, None) == 1
     # O(N*D) extra memory, never O(N^2): doubling N doubles the workspace
     a, b = ctypes.c_size_t(0), ctypes.c_size_t(0)
