@@ -50,6 +50,9 @@ struct DeviceInfo {
     bool init = false;
     bool sm100 = false;
     int sm_count = 0;
+    // clusters of the bf16 forward (index 0: D = 64, 1: D = 128) that can be
+    // resident at once, per cluster size; -1 until first queried
+    int fwd_clusters[2][17];
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -74,6 +77,8 @@ mea_status_t device_info(DeviceInfo** out) {
             return fail(MEA_ERR_CUDA, "cudaDeviceGetAttribute", "failed");
         d.sm100 = (major == 10 && minor == 0);
         d.sm_count = sms;
+        for (auto& row : d.fwd_clusters)
+            for (int& n : row) n = -1;
         d.init = true;
     }
     if (g_encode == nullptr) {
@@ -87,6 +92,15 @@ mea_status_t device_info(DeviceInfo** out) {
     if (!d.sm100) return fail(MEA_ERR_UNSUPPORTED, "device", "compute capability 10.0 (sm_100a) required");
     *out = &d;
     return MEA_OK;
+}
+
+// Clusters of `size` CTAs of the bf16 forward that fit on the device at once
+// (cached; 0 if the query fails, which only disables that cluster size).
+int fwd_max_clusters(DeviceInfo* d, int D, int size) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    int& n = d->fwd_clusters[D == 128 ? 1 : 0][size];
+    if (n < 0) n = mea::fwd_bf16_max_active_clusters(D, size);
+    return n;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -223,12 +237,24 @@ mea_status_t mea_attn_fwd(const void* q, const void* k, const void* v, void* o, 
     a.scale = scale;
     if (BH > 65535) return MEA_ERR_UNSUPPORTED;
     // Split the keys over a cluster when the (query tile x head) grid would
-    // leave most SMs idle, e.g. decode-shaped calls with a handful of rows.
+    // leave more than half of the SMs idle, e.g. decode-shaped calls with a
+    // handful of rows: the cluster size is the one that puts the most CTAs to
+    // work while every cluster of the launch is resident at once (one wave),
+    // with at least two key tiles per CTA.
     {
         const long long base = (long long)((Nq + 255) / 256) * BH;
         const int key_tiles = (Nk + 127) / 128;
         int chunks = 1;
-        while (chunks < 16 && base * chunks * 2 <= dev->sm_count && key_tiles >= chunks * 4) chunks *= 2;
+        if (base * 2 <= dev->sm_count) {
+            long long best = base;
+            for (int c = 2; c <= 16 && key_tiles >= 2 * c; ++c) {
+                if (base > fwd_max_clusters(dev, D, c)) continue;
+                if (base * c > best) {
+                    best = base * c;
+                    chunks = c;
+                }
+            }
+        }
         a.chunks = chunks;
         a.chunk_len = (int)round_up((size_t)((Nk + chunks - 1) / chunks), 128);
         if ((long long)((Nq + 255) / 256) * chunks > 0x7fffffffLL) return MEA_ERR_UNSUPPORTED;

@@ -71,6 +71,7 @@ struct FwdBarriers {
     uint64_t s_full[2];
     uint64_t p_ready[2];
     uint64_t o_final;
+    uint64_t merge_ready;
     uint64_t drain;
     unsigned tmem_base;
     int abort_flag;
@@ -135,6 +136,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&bars->p_ready[t], 128);
         }
         mbar_init(&bars->o_final, 1);
+        mbar_init(&bars->merge_ready, 128);
         mbar_init(&bars->drain, 1);
         bars->abort_flag = 0;
         fence_mbar_init();
@@ -236,18 +238,49 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             };
             uint32_t k_off = 0;
             int k_stage = 0;
-            if (ok && n_kv > 0) ok = next_tile(k_off, k_stage);
-            if (ok && n_kv > 0) {
+            if (!two) {
+                // One live query tile: the two TMEM slots run the recurrence for
+                // the same rows over alternate key tiles (slot t takes tiles
+                // t, t+2, ...), so one slot's softmax overlaps the other's MMAs.
+                // Ring tiles are still taken in the producer's order K_0, V_0,
+                // K_1, V_1, ...; a slot's V tile is held until its P is ready.
+                uint32_t v_off[2] = {0, 0};
+                int v_stage[2] = {0, 0};
+                for (int t = 0; ok && t < 2 && t < n_kv; ++t) {
+                    if (!(ok = next_tile(k_off, k_stage))) break;
+                    tc_fence_after();
+                    issue_s(t ? tS1 : tS0, q_lo0, k_off);
+                    mma_commit(&bars->s_full[t]);
+                    mma_commit(&bars->empty[k_stage]);
+                    ok = next_tile(v_off[t], v_stage[t]);
+                }
+                for (int j = 0; ok && j < n_kv; ++j) {
+                    const int t = j & 1;
+                    const int i = j >> 1;  // iteration of slot t
+                    if (!(ok = mbar_wait(&bars->p_ready[t], i & 1, abort_flag))) break;
+                    tc_fence_after();
+                    issue_pv(t ? tO1 : tO0, t ? tS1 : tS0, v_off[t], i > 0 ? 1u : 0u);
+                    mma_commit(&bars->empty[v_stage[t]]);
+                    if (j + 2 < n_kv) {
+                        if (!(ok = next_tile(k_off, k_stage))) break;
+                        tc_fence_after();
+                        issue_s(t ? tS1 : tS0, q_lo0, k_off);
+                        mma_commit(&bars->s_full[t]);
+                        mma_commit(&bars->empty[k_stage]);
+                        ok = next_tile(v_off[t], v_stage[t]);
+                    }
+                }
+            }
+            if (two && ok && n_kv > 0) ok = next_tile(k_off, k_stage);
+            if (two && ok && n_kv > 0) {
                 tc_fence_after();
                 issue_s(tS0, q_lo0, k_off);
                 mma_commit(&bars->s_full[0]);
-                if (two) {
-                    issue_s(tS1, q_lo1, k_off);
-                    mma_commit(&bars->s_full[1]);
-                }
+                issue_s(tS1, q_lo1, k_off);
+                mma_commit(&bars->s_full[1]);
                 mma_commit(&bars->empty[k_stage]);
             }
-            for (int j = 0; ok && j < n_kv; ++j) {
+            for (int j = 0; two && ok && j < n_kv; ++j) {
                 const bool more = (j + 1 < n_kv);
                 const unsigned acc0 = j > 0 ? 1u : 0u;
                 uint32_t v_off = 0;
@@ -264,17 +297,13 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     mma_commit(&bars->s_full[0]);
                 }
                 // tile 1: O_1 += P_1 V_j, then S_1 = Q_1 K_{j+1}^T
-                if (two) {
-                    if (!(ok = mbar_wait(&bars->p_ready[1], j & 1, abort_flag))) break;
-                    tc_fence_after();
-                    issue_pv(tO1, tS1, v_off, acc0);
-                }
+                if (!(ok = mbar_wait(&bars->p_ready[1], j & 1, abort_flag))) break;
+                tc_fence_after();
+                issue_pv(tO1, tS1, v_off, acc0);
                 mma_commit(&bars->empty[v_stage]);
                 if (more) {
-                    if (two) {
-                        issue_s(tS1, q_lo1, k_off);
-                        mma_commit(&bars->s_full[1]);
-                    }
+                    issue_s(tS1, q_lo1, k_off);
+                    mma_commit(&bars->s_full[1]);
                     mma_commit(&bars->empty[k_stage]);
                 }
             }
@@ -285,148 +314,178 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     } else {
         // ------------------------------------------------ softmax / epilogue
-        const int t = (warp - 2) >> 2;                     // query tile of these four warps
+        const int t = (warp - 2) >> 2;                     // TMEM slot of these four warps
         const unsigned sub = warp & 3;                     // TMEM sub-partition (lanes 32*sub..)
-        const int r = sub * 32 + lane;                     // row within the tile
+        const int r = sub * 32 + lane;                     // row within the query tile
         const unsigned lane_off = (sub * 32u) << 16;
         const unsigned tS = tmem + lane_off + (t ? 128u : 0u);
         const unsigned tO = tmem + lane_off + (t ? 384u : 256u);
+        // With two live query tiles slot t owns query tile t and every key
+        // tile; with one, both slots own query tile 0 and slot t takes the key
+        // tiles t, t+2, ... (merged below).
+        const bool split = !two;
+        const int n_mine = split ? (n_kv + 1 - t) / 2 : n_kv;
+        const int row0 = m0 + (split ? 0 : t * kTileM);
         // Rows at or past Nq are never stored and a row of O depends only on
         // the same row of P, so a warp whose 32 rows all lie past Nq only keeps
-        // the handshake (its P lanes hold whatever S left there), and the warps
-        // of an unused second tile take no part at all.
-        if ((m0 + t * kTileM + (int)sub * 32) >= Nq) {
-            if (t == 0 || two) {
-                for (int j = 0; j < n_kv; ++j) {
-                    if (!mbar_wait(&bars->s_full[t], j & 1, abort_flag)) break;
-                    mbar_arrive(&bars->p_ready[t]);
-                }
-            }
-        } else {
-        const float c_log2 = scale * kLog2e;
+        // the handshake (its P lanes hold whatever S left there).
+        const bool live = (row0 + (int)sub * 32) < Nq;
         float m_ref = -INFINITY;  // reference maximum, base-2 units of scale*s
         float l = 0.f;
         bool ok = true;
-        for (int j = 0; j < n_kv; ++j) {
-            if (!(ok = mbar_wait(&bars->s_full[t], j & 1, abort_flag))) break;
-            tc_fence_after();
-            uint32_t sr[kTileN];
-#pragma unroll
-            for (int c0 = 0; c0 < kTileN; c0 += 32)
-                tmem_ld32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(&sr[c0]));
-            tmem_wait_ld();
-            const int nvalid = c_end - (c_begin + j * kTileN);
-            if (nvalid < kTileN) {
-#pragma unroll
-                for (int c = 0; c < kTileN; ++c)
-                    if (c >= nvalid) sr[c] = __float_as_uint(-INFINITY);
+        if (!live) {
+            for (int i = 0; i < n_mine; ++i) {
+                if (!(ok = mbar_wait(&bars->s_full[t], i & 1, abort_flag))) break;
+                mbar_arrive(&bars->p_ready[t]);
             }
-            // row maximum as 8 independent chains (one thread owns the row, so a
-            // single 128-long dependent chain would dominate the softmax latency)
-            float mxa[8];
+        } else {
+            const float c_log2 = scale * kLog2e;
+            for (int it = 0; it < n_mine; ++it) {
+                const int j = split ? 2 * it + t : it;  // key tile within this CTA's range
+                if (!(ok = mbar_wait(&bars->s_full[t], it & 1, abort_flag))) break;
+                tc_fence_after();
+                uint32_t sr[kTileN];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) mxa[i] = __uint_as_float(sr[i]);
+                for (int c0 = 0; c0 < kTileN; c0 += 32)
+                    tmem_ld32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(&sr[c0]));
+                tmem_wait_ld();
+                const int nvalid = c_end - (c_begin + j * kTileN);
+                if (nvalid < kTileN) {
 #pragma unroll
-            for (int c = 8; c < kTileN; c += 8)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) mxa[i] = fmaxf(mxa[i], __uint_as_float(sr[c + i]));
-            const float mx = fmaxf(fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])),
-                                   fmaxf(fmaxf(mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7])));
-            const float m_blk = mx * c_log2;
-            float m_new = m_ref;
-            bool rescale = false;
-            float alpha = 1.f;
-            if (j == 0) {
-                m_new = m_blk;
-            } else if (__any_sync(0xffffffffu, m_blk - m_ref > kRescaleThreshold)) {
-                // warp-uniform decision: tcgen05.ld/st below are warp-collective
-                m_new = fmaxf(m_ref, m_blk);
-                alpha = ex2_approx(m_ref - m_new);
-                rescale = true;
-            }
-            m_ref = m_new;
-            l *= alpha;
-            // row sum as 8 independent partial sums (same reason as the maximum)
-            float rsa[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) rsa[i] = 0.f;
-#pragma unroll
-            for (int c0 = 0; c0 < kTileN; c0 += 32) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c0 + c]), c_log2, -m_ref));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c0 + c + 1]), c_log2, -m_ref));
-                    rsa[(c / 2) & 7] += p0 + p1;
-                    pk[c / 2] = pack_bf16x2(p0, p1);
+                    for (int c = 0; c < kTileN; ++c)
+                        if (c >= nvalid) sr[c] = __float_as_uint(-INFINITY);
                 }
-                tmem_st16(tS + c0 / 2, pk);
-            }
-            l += ((rsa[0] + rsa[1]) + (rsa[2] + rsa[3])) + ((rsa[4] + rsa[5]) + (rsa[6] + rsa[7]));
-            if (rescale) {
-                // PV_t(j-1) has completed (it was issued before S_t(j), whose
-                // commit we waited on), so O_t can be rescaled in place.
+                // row maximum as 8 independent chains (one thread owns the row, so a
+                // single 128-long dependent chain would dominate the softmax latency)
+                float mxa[8];
 #pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    uint32_t ov[32];
-                    tmem_ld32(tO + c0, ov);
-                    tmem_wait_ld();
+                for (int i = 0; i < 8; ++i) mxa[i] = __uint_as_float(sr[i]);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                    tmem_st32(tO + c0, ov);
+                for (int c = 8; c < kTileN; c += 8)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) mxa[i] = fmaxf(mxa[i], __uint_as_float(sr[c + i]));
+                const float mx = fmaxf(fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])),
+                                       fmaxf(fmaxf(mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7])));
+                const float m_blk = mx * c_log2;
+                float m_new = m_ref;
+                bool rescale = false;
+                float alpha = 1.f;
+                if (it == 0) {
+                    m_new = m_blk;
+                } else if (__any_sync(0xffffffffu, m_blk - m_ref > kRescaleThreshold)) {
+                    // warp-uniform decision: tcgen05.ld/st below are warp-collective
+                    m_new = fmaxf(m_ref, m_blk);
+                    alpha = ex2_approx(m_ref - m_new);
+                    rescale = true;
                 }
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&bars->p_ready[t]);
-        }
-        if (ok && mbar_wait(&bars->o_final, 0, abort_flag)) {
-            tc_fence_after();
-            const int row = m0 + t * kTileM + r;
-            if (nranks == 1) {
-                const float inv_l = 1.f / l;
-                uint16_t* orow = o + ((size_t)bh * Nq + row) * D;
+                m_ref = m_new;
+                l *= alpha;
+                // row sum as 8 independent partial sums (same reason as the maximum)
+                float rsa[8];
 #pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    uint32_t ov[32];
-                    tmem_ld32(tO + c0, ov);
-                    tmem_wait_ld();
-                    if (row < Nq) {
-                        uint32_t packed[16];
+                for (int i = 0; i < 8; ++i) rsa[i] = 0.f;
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            packed[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l,
-                                                    __uint_as_float(ov[2 * i + 1]) * inv_l);
-                        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+                for (int c0 = 0; c0 < kTileN; c0 += 32) {
+                    uint32_t pk[16];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                    for (int c = 0; c < 32; c += 2) {
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c0 + c]), c_log2, -m_ref));
+                        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c0 + c + 1]), c_log2, -m_ref));
+                        rsa[(c / 2) & 7] += p0 + p1;
+                        pk[c / 2] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(tS + c0 / 2, pk);
+                }
+                l += ((rsa[0] + rsa[1]) + (rsa[2] + rsa[3])) + ((rsa[4] + rsa[5]) + (rsa[6] + rsa[7]));
+                if (rescale) {
+                    // PV_t(j-1) has completed (it was issued before S_t(j), whose
+                    // commit we waited on), so O_t can be rescaled in place.
+#pragma unroll
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        uint32_t ov[32];
+                        tmem_ld32(tO + c0, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+                        tmem_st32(tO + c0, ov);
                     }
                 }
-                if (row < Nq) lse[(size_t)bh * Nq + row] = (m_ref + __log2f(l)) * kLn2;
-            } else {
-                // chunk summary of this row for the cluster merge: (m_ref, l) and the
-                // unnormalised accumulator (zero when this CTA's chunk is empty)
-                float* prow = part_row<D>(smem, t, r);
-#pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    uint32_t ov[32];
-                    tmem_ld32(tO + c0, ov);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; i += 4) {
-                        float4 f = (n_kv > 0) ? make_float4(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1]),
-                                                            __uint_as_float(ov[i + 2]), __uint_as_float(ov[i + 3]))
-                                              : make_float4(0.f, 0.f, 0.f, 0.f);
-                        *reinterpret_cast<float4*>(prow + c0 + i) = f;
-                    }
-                }
-                float* ml = part_ml<D>(smem, t, r);
-                ml[0] = (n_kv > 0) ? m_ref : -INFINITY;
-                ml[1] = (n_kv > 0) ? l : 0.f;
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&bars->p_ready[t]);
             }
         }
-        }  // rows of this warp below Nq
+
+        if (split && t == 1) {
+            // hand this slot's (m_ref, l) to slot 0, whose warps read its O
+            // straight from TMEM (same lanes); the merge area is free once the
+            // last MMA has completed
+            if (live && ok && mbar_wait(&bars->o_final, 0, abort_flag)) {
+                float* ml = part_ml<D>(smem, 1, r);
+                ml[0] = m_ref;
+                ml[1] = l;
+            }
+            mbar_arrive(&bars->merge_ready);
+        } else if (live && ok && mbar_wait(&bars->o_final, 0, abort_flag)) {
+            tc_fence_after();
+            const int row = row0 + r;
+            // split mode: fold slot 1's summary of the same rows in with the
+            // two-block formulas (slot 1 is empty when the range has one key tile)
+            const bool with1 = split && n_kv >= 2;
+            float w0 = 1.f, w1 = 0.f, M = m_ref, L = l;
+            if (with1) {
+                ok = mbar_wait(&bars->merge_ready, 0, abort_flag);
+                const float* ml1 = part_ml<D>(smem, 1, r);
+                const float m1 = ml1[0], l1 = ml1[1];
+                M = fmaxf(m_ref, m1);
+                w0 = ex2_approx(m_ref - M);
+                w1 = ex2_approx(m1 - M);
+                L = w0 * l + w1 * l1;
+            }
+            const unsigned tO1 = tmem + lane_off + 384u;
+            const bool has = n_kv > 0;
+            const float inv_L = 1.f / L;
+            uint16_t* orow = o + ((size_t)bh * Nq + row) * D;
+            float* prow = part_row<D>(smem, t, r);
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 16) {
+                uint32_t a0[16], a1[16];
+                tmem_ld16(tO + c0, a0);
+                if (with1) tmem_ld16(tO1 + c0, a1);
+                tmem_wait_ld();
+                float f[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    f[i] = w0 * __uint_as_float(a0[i]);
+                    if (with1) f[i] = fmaf(w1, __uint_as_float(a1[i]), f[i]);
+                }
+                if (!ok || row >= Nq) continue;
+                if (nranks == 1) {
+                    uint32_t packed[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) packed[i] = pack_bf16x2(f[2 * i] * inv_L, f[2 * i + 1] * inv_L);
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+                    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                } else {
+                    // chunk summary of this row for the cluster merge: the
+                    // unnormalised accumulator (zero when this CTA's range is empty)
+#pragma unroll
+                    for (int i = 0; i < 16; i += 4)
+                        *reinterpret_cast<float4*>(prow + c0 + i) =
+                            has ? make_float4(f[i], f[i + 1], f[i + 2], f[i + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+            if (ok && row < Nq) {
+                if (nranks == 1) {
+                    lse[(size_t)bh * Nq + row] = (M + __log2f(L)) * kLn2;
+                } else {
+                    float* ml = part_ml<D>(smem, t, r);
+                    ml[0] = has ? M : -INFINITY;
+                    ml[1] = has ? L : 0.f;
+                }
+            }
+        }
     }
 
     if (nranks > 1) {
@@ -434,53 +493,57 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // on the abort path, so no CTA leaves while another reads its memory
         __syncwarp();
         cluster_sync_all();
-        if (rank == 0 && warp >= 2) {
+        if (warp >= 2 && !*abort_flag) {
+            // The merge is spread over the whole cluster: rank c finishes the
+            // 4-column groups g = c, c + nranks, ... of every row, so each
+            // thread issues all of its remote loads at once and no CTA does
+            // more than its share.
             namespace cg = cooperative_groups;
             cg::cluster_group cluster = cg::this_cluster();
-            const int t = (warp - 2) >> 2;
-            const int r = (warp & 3) * 32 + lane;
-            const int row = m0 + t * kTileM + r;
-            if (row < Nq && !*abort_flag) {
-                float M = -INFINITY;
-                for (unsigned c = 0; c < nranks; ++c) {
-                    const float* ml = cluster.map_shared_rank(part_ml<D>(smem, t, r), c);
-                    M = fmaxf(M, ml[0]);
-                }
-                float L = 0.f;
-                float w[16];
+            constexpr int kGroups = D / 4;
+            const int gpr = (kGroups - (int)rank + (int)nranks - 1) / (int)nranks;  // groups of this rank
+            const int rows = min(2 * kTileM, Nq - m0);
+            const int items = rows * gpr;
+            for (int item = (int)threadIdx.x - 64; item < items; item += kThreads - 64) {
+                const int i = item / gpr;                        // row within this CTA's tile pair
+                const int g = (int)rank + (int)nranks * (item - i * gpr);
+                const int t = i / kTileM;
+                const int r = i - t * kTileM;
+                float mc[16], lc[16];
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
-                    w[c] = 0.f;
+                    mc[c] = -INFINITY;
+                    lc[c] = 0.f;
                     if (c < (int)nranks) {
                         const float* ml = cluster.map_shared_rank(part_ml<D>(smem, t, r), (unsigned)c);
-                        w[c] = ex2_approx(ml[0] - M);     // 0 for empty chunks (m = -inf)
-                        L = fmaf(w[c], ml[1], L);
+                        mc[c] = ml[0];
+                        lc[c] = ml[1];
+                    }
+                }
+                float M = mc[0];
+#pragma unroll
+                for (int c = 1; c < 16; ++c) M = fmaxf(M, mc[c]);
+                float L = 0.f;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    if (c < (int)nranks) {
+                        const float w = ex2_approx(mc[c] - M);   // 0 for empty chunks (m = -inf)
+                        const float* prow = cluster.map_shared_rank(part_row<D>(smem, t, r), (unsigned)c);
+                        const float4 v = *reinterpret_cast<const float4*>(prow + 4 * g);
+                        L = fmaf(w, lc[c], L);
+                        acc.x = fmaf(w, v.x, acc.x);
+                        acc.y = fmaf(w, v.y, acc.y);
+                        acc.z = fmaf(w, v.z, acc.z);
+                        acc.w = fmaf(w, v.w, acc.w);
                     }
                 }
                 const float inv_L = 1.f / L;
+                const int row = m0 + i;
                 uint16_t* orow = o + ((size_t)bh * Nq + row) * D;
-#pragma unroll 1
-                for (int d = 0; d < D; d += 8) {
-                    float acc[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        if (c < (int)nranks) {
-                            const float* prow = cluster.map_shared_rank(part_row<D>(smem, t, r), (unsigned)c);
-                            const float4 a = *reinterpret_cast<const float4*>(prow + d);
-                            const float4 b = *reinterpret_cast<const float4*>(prow + d + 4);
-                            acc[0] = fmaf(w[c], a.x, acc[0]); acc[1] = fmaf(w[c], a.y, acc[1]);
-                            acc[2] = fmaf(w[c], a.z, acc[2]); acc[3] = fmaf(w[c], a.w, acc[3]);
-                            acc[4] = fmaf(w[c], b.x, acc[4]); acc[5] = fmaf(w[c], b.y, acc[5]);
-                            acc[6] = fmaf(w[c], b.z, acc[6]); acc[7] = fmaf(w[c], b.w, acc[7]);
-                        }
-                    }
-                    *reinterpret_cast<uint4*>(orow + d) =
-                        make_uint4(pack_bf16x2(acc[0] * inv_L, acc[1] * inv_L), pack_bf16x2(acc[2] * inv_L, acc[3] * inv_L),
-                                   pack_bf16x2(acc[4] * inv_L, acc[5] * inv_L), pack_bf16x2(acc[6] * inv_L, acc[7] * inv_L));
-                }
-                lse[(size_t)bh * Nq + row] = (M + __log2f(L)) * kLn2;
+                *reinterpret_cast<uint2*>(orow + 4 * g) =
+                    make_uint2(pack_bf16x2(acc.x * inv_L, acc.y * inv_L), pack_bf16x2(acc.z * inv_L, acc.w * inv_L));
+                if (g == 0) lse[(size_t)bh * Nq + row] = (M + __log2f(L)) * kLn2;
             }
         }
         cluster_sync_all();
@@ -525,7 +588,41 @@ cudaError_t launch_d(const Bf16FwdArgs& a, cudaStream_t stream) {
     return cudaLaunchKernelEx(&cfg, kern, a.tm_q, a.tm_k, a.tm_v, a.o, a.lse, a.Nq, a.Nk, a.scale, a.chunk_len);
 }
 
+template <int D>
+int max_active_clusters_d(int cluster) {
+    using Cfg = FwdCfg<D>;
+    auto kern = fwd_bf16_kernel<D>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
+        return 0;
+    if (cluster > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+        return 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cluster, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
+
 }  // namespace
+
+int fwd_bf16_max_active_clusters(int D, int cluster) {
+    if (cluster < 1 || cluster > 16) return 0;
+    if (D == 64) return max_active_clusters_d<64>(cluster);
+    if (D == 128) return max_active_clusters_d<128>(cluster);
+    return 0;
+}
 
 cudaError_t launch_fwd_bf16(const Bf16FwdArgs& a, cudaStream_t stream) {
     if (a.D == 64) return launch_d<64>(a, stream);

@@ -56,6 +56,9 @@ struct Bf16FwdArgs {
     int chunk_len;  // keys per chunk (multiple of 128) when chunks > 1
 };
 cudaError_t launch_fwd_bf16(const Bf16FwdArgs& a, cudaStream_t stream);
+// Clusters of `cluster` CTAs of the bf16 forward for head dim D that can be
+// resident at once (cudaOccupancyMaxActiveClusters); 0 on failure.
+int fwd_bf16_max_active_clusters(int D, int cluster);
 
 // bf16 backward (bwd_bf16.cu).
 struct Bf16BwdArgs {

@@ -13,7 +13,7 @@ import torch
 
 import oracle
 from synthetic_inputs import custom, make_inputs, make_workload, to_f64
-from tests._parity import BF16_O, assert_close, assert_lse_close, to_np
+from tests._parity import BF16_GRAD, BF16_O, assert_close, assert_lse_close, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -144,3 +144,24 @@ def test_deterministic():
     a, la = gpu_fwd(q, k, v, w.scale)
     b, lb = gpu_fwd(q, k, v, w.scale)
     assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 300, 400, 64), (1, 1, 1, 5000, 128), (1, 2, 129, 700, 128)])
+def test_single_tile_split_repeat(shape):
+    """CTAs whose rows fit in one query tile split their keys over both TMEM slots and merge the
+    two summaries; repeat forward + backward 20 times against the oracle (a race would show as a
+    sporadic wrong or non-finite value)."""
+    import exact_memory_efficient_b200 as m
+    w = custom(*shape, "bf16")
+    q, k, v, do = make_inputs(w, 11)
+    qd, kd, vd, dod = (x.cuda() for x in (q, k, v, do))
+    rq, rk, rv, ro, rl = oracle.attention_backward(to_f64(q), to_f64(k), to_f64(v), to_f64(do), w.scale)
+    for _ in range(20):
+        o, lse = m.attention_forward(qd, kd, vd, w.scale)
+        dq, dk, dv = m.attention_backward(qd, kd, vd, o, lse, dod, w.scale)
+        assert m.mea_last_device_error() == m.MEA_OK
+        assert_close(to_np(o), ro, *BF16_O, what=f"O {shape}")
+        assert_lse_close(to_np(lse), rl, to_f64(q), to_f64(k), w.scale, what=f"lse {shape}")
+        assert_close(to_np(dq), rq, *BF16_GRAD, what=f"dQ {shape}", bf16_output=True)
+        assert_close(to_np(dk), rk, *BF16_GRAD, what=f"dK {shape}", bf16_output=True)
+        assert_close(to_np(dv), rv, *BF16_GRAD, what=f"dV {shape}", bf16_output=True)
