@@ -355,17 +355,20 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     for (int c = 0; c < kTileN; ++c)
                         if (c >= nvalid) sr[c] = __float_as_uint(-INFINITY);
                 }
-                // row maximum as 8 independent chains (one thread owns the row, so a
-                // single 128-long dependent chain would dominate the softmax latency)
+                // row maximum as 8 independent chains of 3-input maxima (one thread
+                // owns the row, so a single 128-long dependent chain would dominate
+                // the softmax latency; the softmax warps are issue-bound, so each
+                // instruction should retire two new values)
                 float mxa[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) mxa[i] = __uint_as_float(sr[i]);
+                for (int i = 0; i < 8; ++i) mxa[i] = fmaxf(__uint_as_float(sr[i]), __uint_as_float(sr[8 + i]));
 #pragma unroll
-                for (int c = 8; c < kTileN; c += 8)
+                for (int c = 16; c < kTileN; c += 16)
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) mxa[i] = fmaxf(mxa[i], __uint_as_float(sr[c + i]));
-                const float mx = fmaxf(fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])),
-                                       fmaxf(fmaxf(mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7])));
+                    for (int i = 0; i < 8; ++i)
+                        mxa[i] = fmax3(mxa[i], __uint_as_float(sr[c + i]), __uint_as_float(sr[c + 8 + i]));
+                const float mx = fmaxf(fmax3(mxa[0], mxa[1], mxa[2]),
+                                       fmax3(fmax3(mxa[3], mxa[4], mxa[5]), mxa[6], mxa[7]));
                 const float m_blk = mx * c_log2;
                 float m_new = m_ref;
                 bool rescale = false;
