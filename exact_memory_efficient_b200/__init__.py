@@ -28,7 +28,8 @@ __all__ = [
     "MEA_ERR_CUDA", "MEA_ERR_TIMEOUT", "MEA_DTYPE_F32", "MEA_DTYPE_BF16",
     "MEA_BWD_ALL", "MEA_BWD_PREPROCESS", "MEA_BWD_MAIN", "MEA_BWD_FINALIZE",
     "mea_attn_fwd", "mea_attn_bwd", "mea_attn_bwd_phase", "mea_attn_bwd_workspace_size", "mea_attn_bwd_noalloc",
-    "mea_attn_fwd_gqa", "mea_attn_bwd_gqa", "mea_attn_bwd_gqa_workspace_size", "mea_last_device_error",
+    "mea_attn_fwd_gqa", "mea_attn_bwd_gqa", "mea_attn_bwd_gqa_workspace_size", "mea_attn_fwd_fp8",
+    "mea_last_device_error",
     "mea_selftest_bounded_wait", "mea_status_string", "mea_last_error_message", "mea_version", "attention_forward", "attention_backward",
 ]
 
@@ -92,6 +93,8 @@ def load_library() -> ctypes.CDLL:
     lib.mea_attn_bwd_gqa_workspace_size.restype = i
     lib.mea_attn_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, sz, vp]
     lib.mea_attn_bwd_gqa.restype = i
+    lib.mea_attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, f, vp]
+    lib.mea_attn_fwd_fp8.restype = i
     lib.mea_selftest_bounded_wait.argtypes = [vp, vp]
     lib.mea_selftest_bounded_wait.restype = i
     lib.mea_last_device_error.argtypes = [vp]
@@ -253,6 +256,23 @@ def mea_attn_bwd_gqa(q, k, v, o, lse, do, dq, dk, dv, scale: float, workspace, s
                                           _ptr(dk), _ptr(dv), B, H, Hkv, Nq, Nk, D, float(scale), _dtype_code(q),
                                           _ptr(workspace), ws_bytes, _stream_handle(stream))
     _check(st, "mea_attn_bwd_gqa")
+
+
+def mea_attn_fwd_fp8(q, k, v, o, lse, scale: float, q_descale: float, k_descale: float, stream=None) -> None:
+    """C ``mea_attn_fwd_fp8``: q [B,H,Nq,128] and k [B,H_kv,Nk,128] e4m3 (torch.float8_e4m3fn),
+    v [B,H_kv,Nk,128] bf16; writes o [B,H,Nq,128] bf16 and lse [B,H,Nq] fp32."""
+    B, H, Hkv, Nq, Nk, D = _gqa_shapes(q, k, "mea_attn_fwd_fp8")
+    if q.dtype != torch.float8_e4m3fn or k.dtype != torch.float8_e4m3fn:
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_fwd_fp8: q and k must be float8_e4m3fn")
+    if v.dtype != torch.bfloat16 or o.dtype != torch.bfloat16:
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_fwd_fp8: v and o must be bfloat16")
+    if tuple(v.shape) != tuple(k.shape) or tuple(o.shape) != tuple(q.shape):
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_fwd_fp8: shape mismatch")
+    if tuple(lse.shape) != (B, H, Nq) or lse.dtype != torch.float32:
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_fwd_fp8: lse must be fp32 [B, H, Nq]")
+    st = load_library().mea_attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Nq, Nk, D,
+                                          float(scale), float(q_descale), float(k_descale), _stream_handle(stream))
+    _check(st, "mea_attn_fwd_fp8")
 
 
 def mea_selftest_bounded_wait(gave_up, stream=None) -> None:

@@ -50,9 +50,10 @@ struct DeviceInfo {
     bool init = false;
     bool sm100 = false;
     int sm_count = 0;
-    // clusters of the bf16 forward (index 0: D = 64, 1: D = 128) that can be
-    // resident at once, per cluster size; -1 until first queried
-    int fwd_clusters[2][17];
+    // clusters of the tensor-core forward (index 0: D = 64, 1: D = 128,
+    // 2: D = 128 with e4m3 Q/K) that can be resident at once, per cluster
+    // size; -1 until first queried
+    int fwd_clusters[3][17];
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -96,10 +97,10 @@ mea_status_t device_info(DeviceInfo** out) {
 
 // Clusters of `size` CTAs of the bf16 forward that fit on the device at once
 // (cached; 0 if the query fails, which only disables that cluster size).
-int fwd_max_clusters(DeviceInfo* d, int D, int size) {
+int fwd_max_clusters(DeviceInfo* d, int D, bool fp8, int size) {
     std::lock_guard<std::mutex> lk(g_mu);
-    int& n = d->fwd_clusters[D == 128 ? 1 : 0][size];
-    if (n < 0) n = mea::fwd_bf16_max_active_clusters(D, size);
+    int& n = d->fwd_clusters[fp8 ? 2 : (D == 128 ? 1 : 0)][size];
+    if (n < 0) n = mea::fwd_bf16_max_active_clusters(D, fp8, size);
     return n;
 }
 
@@ -125,6 +126,24 @@ mea_status_t make_map(CUtensorMap* m, const void* base, int BH, int N, int D) {
     return MEA_OK;
 }
 
+// 3-D e4m3 map over [BH][N][D] with D = 128: dims {128, N, BH}, box {128, 128, 1}
+// (one 128-byte row per element row), 128-byte swizzle, out-of-range rows read as zero.
+mea_status_t make_map_u8(CUtensorMap* m, const void* base, int BH, int N, int D) {
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D, (cuuint64_t)N * D};
+    cuuint32_t box[3] = {128, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        char buf[64];
+        std::snprintf(buf, sizeof(buf), "CUresult %d (e4m3)", (int)r);
+        return fail(MEA_ERR_CUDA, "cuTensorMapEncodeTiled", buf);
+    }
+    return MEA_OK;
+}
+
 // 3-D fp32 map over the dQ accumulator [BH][Nq][D]: box {32, 64, 1}, no swizzle
 // (target of the backward's TMA reduce-adds; x offsets are multiples of 32 floats).
 mea_status_t make_map_f32_acc(CUtensorMap* m, void* base, int BH, int Nq, int D) {
@@ -143,6 +162,54 @@ mea_status_t make_map_f32_acc(CUtensorMap* m, void* base, int BH, int Nq, int D)
     return MEA_OK;
 }
 
+mea_status_t cuda_status(cudaError_t e, const char* where) {
+    return e == cudaSuccess ? MEA_OK : fail_cuda(where, e);
+}
+
+// The tensor-core forward over BH heads: bf16 q, k (fp8 = false) or e4m3 q, k
+// (fp8 = true, D = 128); bf16 v, o.  Arguments are validated by the caller.
+mea_status_t tc_forward(const void* q, const void* k, const void* v, void* o, float* lse, int BH, int Nq, int Nk,
+                        int D, float scale, bool fp8, DeviceInfo* dev, cudaStream_t s) {
+    mea::Bf16FwdArgs a;
+    mea_status_t st;
+    a.fp8_qk = fp8;
+    if ((st = (fp8 ? make_map_u8 : make_map)(&a.tm_q, q, BH, Nq, D)) != MEA_OK) return st;
+    if ((st = (fp8 ? make_map_u8 : make_map)(&a.tm_k, k, BH, Nk, D)) != MEA_OK) return st;
+    if ((st = make_map(&a.tm_v, v, BH, Nk, D)) != MEA_OK) return st;
+    a.o = static_cast<uint16_t*>(o);
+    a.lse = lse;
+    a.BH = BH;
+    a.Nq = Nq;
+    a.Nk = Nk;
+    a.D = D;
+    a.scale = scale;
+    if (BH > 65535) return MEA_ERR_UNSUPPORTED;
+    // Split the keys over a cluster when the (query tile x head) grid would
+    // leave more than half of the SMs idle, e.g. decode-shaped calls with a
+    // handful of rows: the cluster size is the one that puts the most CTAs to
+    // work while every cluster of the launch is resident at once (one wave),
+    // with at least two key tiles per CTA.
+    {
+        const long long base = (long long)((Nq + 255) / 256) * BH;
+        const int key_tiles = (Nk + 127) / 128;
+        int chunks = 1;
+        if (base * 2 <= dev->sm_count) {
+            long long best = base;
+            for (int c = 2; c <= 16 && key_tiles >= 2 * c; ++c) {
+                if (base > fwd_max_clusters(dev, D, fp8, c)) continue;
+                if (base * c > best) {
+                    best = base * c;
+                    chunks = c;
+                }
+            }
+        }
+        a.chunks = chunks;
+        a.chunk_len = (int)round_up((size_t)((Nk + chunks - 1) / chunks), 128);
+        if ((long long)((Nq + 255) / 256) * chunks > 0x7fffffffLL) return MEA_ERR_UNSUPPORTED;
+    }
+    return cuda_status(mea::launch_fwd_bf16(a, s), "fwd_bf16 launch");
+}
+
 mea_status_t common_checks(int B, int H, int Nq, int Nk, int D, float scale, mea_dtype_t dtype) {
     if (dtype != MEA_DTYPE_F32 && dtype != MEA_DTYPE_BF16) return MEA_ERR_INVALID_ARG;
     if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || D <= 0) return MEA_ERR_INVALID_ARG;
@@ -155,9 +222,6 @@ mea_status_t common_checks(int B, int H, int Nq, int Nk, int D, float scale, mea
     return MEA_OK;
 }
 
-mea_status_t cuda_status(cudaError_t e, const char* where) {
-    return e == cudaSuccess ? MEA_OK : fail_cuda(where, e);
-}
 
 }  // namespace
 
@@ -224,42 +288,7 @@ mea_status_t mea_attn_fwd(const void* q, const void* k, const void* v, void* o, 
         return cuda_status(mea::launch_fwd_f32(a, s), "fwd_f32 launch");
     }
 
-    mea::Bf16FwdArgs a;
-    if ((st = make_map(&a.tm_q, q, BH, Nq, D)) != MEA_OK) return st;
-    if ((st = make_map(&a.tm_k, k, BH, Nk, D)) != MEA_OK) return st;
-    if ((st = make_map(&a.tm_v, v, BH, Nk, D)) != MEA_OK) return st;
-    a.o = static_cast<uint16_t*>(o);
-    a.lse = lse;
-    a.BH = BH;
-    a.Nq = Nq;
-    a.Nk = Nk;
-    a.D = D;
-    a.scale = scale;
-    if (BH > 65535) return MEA_ERR_UNSUPPORTED;
-    // Split the keys over a cluster when the (query tile x head) grid would
-    // leave more than half of the SMs idle, e.g. decode-shaped calls with a
-    // handful of rows: the cluster size is the one that puts the most CTAs to
-    // work while every cluster of the launch is resident at once (one wave),
-    // with at least two key tiles per CTA.
-    {
-        const long long base = (long long)((Nq + 255) / 256) * BH;
-        const int key_tiles = (Nk + 127) / 128;
-        int chunks = 1;
-        if (base * 2 <= dev->sm_count) {
-            long long best = base;
-            for (int c = 2; c <= 16 && key_tiles >= 2 * c; ++c) {
-                if (base > fwd_max_clusters(dev, D, c)) continue;
-                if (base * c > best) {
-                    best = base * c;
-                    chunks = c;
-                }
-            }
-        }
-        a.chunks = chunks;
-        a.chunk_len = (int)round_up((size_t)((Nk + chunks - 1) / chunks), 128);
-        if ((long long)((Nq + 255) / 256) * chunks > 0x7fffffffLL) return MEA_ERR_UNSUPPORTED;
-    }
-    return cuda_status(mea::launch_fwd_bf16(a, s), "fwd_bf16 launch");
+    return tc_forward(q, k, v, o, lse, BH, Nq, Nk, D, scale, false, dev, s);
 }
 
 mea_status_t mea_attn_bwd_workspace_size(int B, int H, int Nq, int Nk, int D, mea_dtype_t dtype, size_t* bytes) {
@@ -402,6 +431,29 @@ mea_status_t mea_attn_fwd_gqa(const void* q, const void* k, const void* v, void*
     mea_status_t st = gqa_rows(H, H_kv, Nq, &rows);
     if (st != MEA_OK) return st;
     return mea_attn_fwd(q, k, v, o, lse, B, H_kv, rows, Nk, D, scale, dtype, stream);
+}
+
+mea_status_t mea_attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                              int H_kv, int Nq, int Nk, int D, float scale, float q_descale, float k_descale,
+                              void* stream) {
+    int rows = 0;
+    mea_status_t st = gqa_rows(H, H_kv, Nq, &rows);
+    if (st != MEA_OK) return st;
+    if (!std::isfinite(q_descale) || !std::isfinite(k_descale) || !(q_descale > 0.f) || !(k_descale > 0.f))
+        return fail(MEA_ERR_INVALID_ARG, "mea_attn_fwd_fp8", "descale factors must be finite and positive");
+    if ((st = common_checks(B, H_kv, rows, Nk, D, scale, MEA_DTYPE_BF16)) != MEA_OK) return st;
+    if (D != 128) return fail(MEA_ERR_UNSUPPORTED, "mea_attn_fwd_fp8", "head dim 128 only");
+    if ((long long)B * H_kv * rows == 0) return MEA_OK;
+    if (Nk == 0) return MEA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !o || !lse) return MEA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse)) return MEA_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    if ((st = device_info(&dev)) != MEA_OK) return st;
+    // the product of e4m3 values is exact in the fp32 accumulator, so the
+    // descale factors fold into the softmax scale
+    const float eff = scale * q_descale * k_descale;
+    if (!std::isfinite(eff)) return MEA_ERR_INVALID_ARG;
+    return tc_forward(q, k, v, o, lse, B * H_kv, rows, Nk, D, eff, true, dev, static_cast<cudaStream_t>(stream));
 }
 
 mea_status_t mea_attn_bwd_gqa_workspace_size(int B, int H, int H_kv, int Nq, int Nk, int D, mea_dtype_t dtype,

@@ -54,12 +54,18 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
 
-template <int D>
+// F8: Q and K are e4m3 (one byte per element) and S = Q K^T runs as
+// kind::f8f6f4; V, P and O stay bf16.
+template <int D, bool F8 = false>
 struct FwdCfg {
-    static constexpr int kTileBytes = kTileN * D * 2;         // one K or V tile
-    static constexpr int kQBytes = kTileM * D * 2;            // one Q tile
-    static constexpr int kStages = (D == 128) ? 4 : 6;
-    static constexpr int kBoxBytes = 128 * 128;               // one 64-column box of 128 rows
+    static constexpr int kQKElem = F8 ? 1 : 2;                // bytes per Q/K element
+    static constexpr int kQKBox = 128 / kQKElem;              // Q/K elements per 128-byte box row
+    static constexpr int kKBytes = kTileN * D * kQKElem;      // one K tile
+    static constexpr int kVBytes = kTileN * D * 2;            // one V tile
+    static constexpr int kTileBytes = kVBytes;                // one ring stage (a K tile uses its start)
+    static constexpr int kQBytes = kTileM * D * kQKElem;      // one Q tile
+    static constexpr int kStages = F8 ? ((D == 128) ? 5 : 7) : ((D == 128) ? 4 : 6);
+    static constexpr int kBoxBytes = 128 * 128;               // one 128-byte-wide box of 128 rows
     static constexpr int kSmemData = 2 * kQBytes + kStages * kTileBytes;
     static constexpr int kSmemBytes = kSmemData + 1024 /*barriers*/ + 1024 /*alignment slack*/;
 };
@@ -89,18 +95,19 @@ __device__ __forceinline__ float* part_ml(uint8_t* smem, int t, int r) {
     return reinterpret_cast<float*>(smem) + (size_t)2 * kTileM * (D + 4) + ((size_t)t * kTileM + r) * 2;
 }
 static_assert(2 * 128 * (128 + 4) * 4 + 2 * 128 * 2 * 4 <= FwdCfg<128>::kSmemData, "merge area (D=128)");
+static_assert(2 * 128 * (128 + 4) * 4 + 2 * 128 * 2 * 4 <= FwdCfg<128, true>::kSmemData, "merge area (D=128, fp8)");
 static_assert(2 * 128 * (64 + 4) * 4 + 2 * 128 * 2 * 4 <= FwdCfg<64>::kSmemData, "merge area (D=64)");
 
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-template <int D>
+template <int D, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ o,
                 float* __restrict__ lse, int Nq, int Nk, float scale, int chunk_len) {
-    using Cfg = FwdCfg<D>;
+    using Cfg = FwdCfg<D, F8>;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment of the shared-memory address (not of the generic
     // pointer: in a cluster launch each CTA's shared window can sit at a
@@ -160,9 +167,9 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int n_qt = two ? 2 : 1;
             mbar_arrive_expect_tx(&bars->q_full, n_qt * Cfg::kQBytes);
             for (int t = 0; t < n_qt; ++t)
-                for (int b = 0; b < D / 64; ++b)
+                for (int b = 0; b < D / Cfg::kQKBox; ++b)
                     tma_load_3d(sQ + t * Cfg::kQBytes + b * Cfg::kBoxBytes, &tm_q, &bars->q_full,
-                                b * 64, m0 + t * kTileM, bh);
+                                b * Cfg::kQKBox, m0 + t * kTileM, bh);
             const int n_tiles = 2 * n_kv;
             int issued = 0;
             for (int c = 0; c < n_tiles; ++c) {
@@ -171,11 +178,13 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (!mbar_wait(&bars->empty[s], ((c / Cfg::kStages) - 1) & 1, abort_flag)) break;
                 }
                 uint8_t* dst = sRing + s * Cfg::kTileBytes;
-                const CUtensorMap* tm = (c & 1) ? &tm_v : &tm_k;
+                const bool is_v = c & 1;
+                const CUtensorMap* tm = is_v ? &tm_v : &tm_k;
                 const int key0 = c_begin + (c >> 1) * kTileN;
-                mbar_arrive_expect_tx(&bars->full[s], Cfg::kTileBytes);
-                for (int b = 0; b < D / 64; ++b)
-                    tma_load_3d(dst + b * Cfg::kBoxBytes, tm, &bars->full[s], b * 64, key0, bh);
+                const int bw = is_v ? 64 : Cfg::kQKBox;               // elements per box row
+                mbar_arrive_expect_tx(&bars->full[s], is_v ? Cfg::kVBytes : Cfg::kKBytes);
+                for (int b = 0; b < D / bw; ++b)
+                    tma_load_3d(dst + b * Cfg::kBoxBytes, tm, &bars->full[s], b * bw, key0, bh);
                 issued = c + 1;
             }
             // Never leave with copies in flight: wait until the last loads landed.
@@ -209,9 +218,18 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 return true;
             };
             auto issue_s = [&](unsigned tS, uint32_t q_lo, uint32_t k_off) {
+                if constexpr (F8) {
+                    // K = 32 e4m3 elements per instruction: the same 32-byte step
+                    constexpr unsigned idesc_s8 = make_idesc_e4m3(128, kTileN);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_ss_lo(tS, q_lo + kmajor_step(kk), ring_k_lo + k_off + kmajor_step(kk), idesc_s, kk > 0);
+                    for (int kk = 0; kk < D / 32; ++kk)
+                        mma_ss_lo_f8(tS, q_lo + kmajor_step(kk), ring_k_lo + k_off + kmajor_step(kk), idesc_s8,
+                                     kk > 0);
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ss_lo(tS, q_lo + kmajor_step(kk), ring_k_lo + k_off + kmajor_step(kk), idesc_s, kk > 0);
+                }
             };
             // In a cluster launch (key split) P V is issued per 64-column block of V,
             // each block addressed by its start address: on this part, an MMA on
@@ -560,10 +578,10 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
 }
 
-template <int D>
+template <int D, bool F8>
 cudaError_t launch_d(const Bf16FwdArgs& a, cudaStream_t stream) {
-    using Cfg = FwdCfg<D>;
-    auto kern = fwd_bf16_kernel<D>;
+    using Cfg = FwdCfg<D, F8>;
+    auto kern = fwd_bf16_kernel<D, F8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int q_tiles = (a.Nq + 2 * kTileM - 1) / (2 * kTileM);
@@ -591,10 +609,10 @@ cudaError_t launch_d(const Bf16FwdArgs& a, cudaStream_t stream) {
     return cudaLaunchKernelEx(&cfg, kern, a.tm_q, a.tm_k, a.tm_v, a.o, a.lse, a.Nq, a.Nk, a.scale, a.chunk_len);
 }
 
-template <int D>
+template <int D, bool F8>
 int max_active_clusters_d(int cluster) {
-    using Cfg = FwdCfg<D>;
-    auto kern = fwd_bf16_kernel<D>;
+    using Cfg = FwdCfg<D, F8>;
+    auto kern = fwd_bf16_kernel<D, F8>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
         return 0;
     if (cluster > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
@@ -620,16 +638,18 @@ int max_active_clusters_d(int cluster) {
 
 }  // namespace
 
-int fwd_bf16_max_active_clusters(int D, int cluster) {
+int fwd_bf16_max_active_clusters(int D, bool fp8_qk, int cluster) {
     if (cluster < 1 || cluster > 16) return 0;
-    if (D == 64) return max_active_clusters_d<64>(cluster);
-    if (D == 128) return max_active_clusters_d<128>(cluster);
+    if (fp8_qk) return D == 128 ? max_active_clusters_d<128, true>(cluster) : 0;
+    if (D == 64) return max_active_clusters_d<64, false>(cluster);
+    if (D == 128) return max_active_clusters_d<128, false>(cluster);
     return 0;
 }
 
 cudaError_t launch_fwd_bf16(const Bf16FwdArgs& a, cudaStream_t stream) {
-    if (a.D == 64) return launch_d<64>(a, stream);
-    if (a.D == 128) return launch_d<128>(a, stream);
+    if (a.fp8_qk) return a.D == 128 ? launch_d<128, true>(a, stream) : cudaErrorInvalidValue;
+    if (a.D == 64) return launch_d<64, false>(a, stream);
+    if (a.D == 128) return launch_d<128, false>(a, stream);
     return cudaErrorInvalidValue;
 }
 

@@ -299,6 +299,20 @@ __device__ __forceinline__ void mma_ss_lo(unsigned d_tmem, uint32_t a_lo, uint32
         ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(kDescHiSw128), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// The same for 8-bit operands (kind::f8f6f4): both from shared memory, one
+// instruction consumes K = 32 elements (32 bytes of each K-major row, the same
+// byte step as K = 16 of bf16).
+__device__ __forceinline__ void mma_ss_lo_f8(unsigned d_tmem, uint32_t a_lo, uint32_t b_lo, unsigned idesc,
+                                             unsigned accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+        "mov.b64 da, {%1, %3};\n\t"
+        "mov.b64 db, {%2, %3};\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], da, db, %4, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(kDescHiSw128), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 // D[tmem] (+)= A[tmem] * B[smem]^T with the B descriptor given by its low word.
 __device__ __forceinline__ void mma_ts_lo(unsigned d_tmem, unsigned a_tmem, uint32_t b_lo, unsigned idesc,
                                           unsigned accumulate) {
@@ -318,6 +332,12 @@ __host__ __device__ constexpr unsigned make_idesc_bf16(unsigned M, unsigned N, u
                                                        unsigned b_mn_major) {
     return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn_major << 15) | (b_mn_major << 16) |
            ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// Instruction descriptor for kind::f8f6f4 with e4m3 A and B (format code 0 in
+// bits 7-9 and 10-12), both K-major, and fp32 D; other fields as above.
+__host__ __device__ constexpr unsigned make_idesc_e4m3(unsigned M, unsigned N) {
+    return (1u << 4) | (0u << 7) | (0u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
 // -------------------------------------------------------------- numerics

@@ -193,6 +193,34 @@ mea_status_t mea_attn_bwd_gqa(const void* q, const void* k, const void* v,
                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Forward pass with e4m3 (FP8) queries and keys.
+ *
+ * Source: "当注意力成为瓶颈从on困境到线性复杂度的技术突围" (section
+ * IO感知：重新审视硬件, the FlashAttention-3 paragraph on FP8 tensor cores).
+ * Reading adopted: Q and K are stored as e4m3 with one dequantisation factor
+ * each (q = q_descale * q8, k = k_descale * k8); V, the probabilities P and
+ * the output stay bf16.  The operation is then exactly that of mea_attn_fwd
+ * on the dequantised inputs:
+ *     O = softmax(scale * q_descale * k_descale * q8 k8^T) v,
+ *     lse_i = ln sum_j exp(scale * q_descale * k_descale * q8_i . k8_j).
+ * S = q8 k8^T runs on the tensor cores as kind::f8f6f4 (each product of two
+ * e4m3 values is exact in the fp32 accumulator); the rest is the bf16 path.
+ *
+ * q: e4m3 [B, H, Nq, D];  k: e4m3 [B, H_kv, Nk, D];  v: bf16 [B, H_kv, Nk, D];
+ * o: bf16 [B, H, Nq, D];  lse: fp32 [B, H, Nq].  H_kv key/value heads are
+ * shared by groups of H / H_kv query heads as in mea_attn_fwd_gqa (H_kv = H is
+ * ordinary multi-head attention).  D = 128 only.  Pointers as for
+ * mea_attn_fwd (16-byte aligned, lse 4-byte aligned).
+ * Errors: MEA_ERR_INVALID_ARG (also for descale factors that are not finite
+ * and positive), MEA_ERR_UNSUPPORTED (D != 128), MEA_ERR_MISALIGNED,
+ * MEA_ERR_CUDA.
+ */
+mea_status_t mea_attn_fwd_fp8(const void* q, const void* k, const void* v,
+                              void* o, float* lse,
+                              int B, int H, int H_kv, int Nq, int Nk, int D, float scale,
+                              float q_descale, float k_descale, void* stream);
+
+/*
  * Backward pass that allocates nothing and takes no workspace.  The paper has
  * no counterpart: this is a deployment convenience of this library.
  *

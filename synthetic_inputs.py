@@ -117,6 +117,45 @@ def make_inputs(w: Workload, seed: int, with_grad_output: bool | None = None):
     return q, k, v, do
 
 
+E4M3_MAX = 448.0  # largest finite value of float8 e4m3 (the "fn" variant without infinities)
+
+
+def make_inputs_fp8(w: Workload, seed: int):
+    """Inputs for the FP8 forward: (q8, k8, v, q_descale, k_descale).
+
+    Same draws as ``make_inputs`` (Q, K, V in fp32 from the same generator
+    order, scaled by ``qk_mult``); Q and K are then quantised per tensor to
+    e4m3: descale = max|x| / 448, x8 = e4m3(x / descale) with round to nearest
+    even (clamped to +-448 first).  V is cast to bf16.  The dequantised values
+    descale * x8 are what the method computes on; the oracle takes their exact
+    fp64 upcast.
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    q = torch.randn((w.B, w.H, w.Nq, w.D), generator=g, dtype=torch.float32)
+    k = torch.randn((w.B, w.H_kv, w.Nk, w.D), generator=g, dtype=torch.float32)
+    v = torch.randn((w.B, w.H_kv, w.Nk, w.D), generator=g, dtype=torch.float32)
+    if w.qk_mult != 1.0:
+        q = q * w.qk_mult
+        k = k * w.qk_mult
+
+    def quant(x):
+        amax = float(x.abs().max()) if x.numel() else 0.0
+        # an fp32 number, as the library takes it
+        descale = float(torch.tensor(amax / E4M3_MAX if amax > 0 else 1.0, dtype=torch.float32))
+        x8 = (x / descale).clamp(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn).contiguous()
+        return x8, descale
+
+    q8, qd = quant(q)
+    k8, kd = quant(k)
+    return q8, k8, v.to(torch.bfloat16).contiguous(), qd, kd
+
+
+def dequant_f64(x8: torch.Tensor, descale: float):
+    """Exact fp64 value of descale * x8 (both factors are exactly representable)."""
+    return x8.to(torch.float64).numpy() * float(descale)
+
+
 def to_f64(t: torch.Tensor):
     """Exact fp64 upcast as a numpy array (bf16 and fp32 values are exactly representable)."""
     return t.detach().to(torch.float64).cpu().numpy()

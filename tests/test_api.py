@@ -167,3 +167,19 @@ def test_gqa_argument_validation(lib):
     assert lib.mea_attn_bwd_gqa_workspace_size(2, 32, 8, 100, 300, 128, BF16, ctypes.byref(out)) == 0
     assert lib.mea_attn_bwd_workspace_size(2, 32, 100, 300, 128, BF16, ctypes.byref(ref)) == 0
     assert out.value == ref.value
+
+
+def test_fp8_argument_validation(lib):
+    def fwd8(D=128, qd=1.0, kd=1.0, H=4, Hkv=2, q=A, Nq=16):
+        return lib.mea_attn_fwd_fp8(q, A, A, A, A, 1, H, Hkv, Nq, 16, D, ctypes.c_float(0.125), ctypes.c_float(qd),
+                                    ctypes.c_float(kd), None)
+
+    assert fwd8(D=64) == 2                 # head dim 128 only
+    assert fwd8(qd=0.0) == 1
+    assert fwd8(kd=-1.0) == 1
+    assert fwd8(qd=float("nan")) == 1
+    assert fwd8(kd=float("inf")) == 1
+    assert fwd8(Hkv=3) == 1                # H not a multiple of H_kv
+    assert fwd8(q=None) == 1
+    assert fwd8(q=A + 8) == 3
+    assert fwd8(Nq=0) == 0                 # no rows: no-op
