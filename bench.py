@@ -35,7 +35,7 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
-from synthetic_inputs import make_inputs, make_workload, custom  # noqa: E402
+from synthetic_inputs import make_inputs, make_inputs_fp8, make_workload, custom  # noqa: E402
 
 WORKLOAD = "long_16384_bf16"
 METRIC = "attention fwd & fwd+bwd TFLOP/s, bf16 n=16384, % of B200 dense BF16 peak"
@@ -435,6 +435,30 @@ def run_ours(args):
                                   "frac_of_peak": round(wg.bwd_flops() / (b_ms * 1e-3) / 1e12 / peak, 3),
                                   "note": f"mean of {reps}; inputs ({wg.H}+2x{wg.H_kv} heads) fit in L2"}
         del qg, kg, vg, dog, og, lg, wsg, grads
+        # FP8 forward (e4m3 Q, K; bf16 V, O) on the step's workload
+        q8, k8, v8, qd8, kd8 = make_inputs_fp8(w, 0)
+        q8, k8, v8 = q8.to(dev), k8.to(dev), v8.to(dev)
+        o8 = torch.empty((w.B, w.H, w.Nq, w.D), dtype=torch.bfloat16, device=dev)
+        l8 = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+        for _ in range(3):
+            m.mea_attn_fwd_fp8(q8, k8, v8, o8, l8, scale, qd8, kd8)
+        reps = 10
+        ev8 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for e0, e1 in ev8:
+            e0.record(stream)
+            m.mea_attn_fwd_fp8(q8, k8, v8, o8, l8, scale, qd8, kd8)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        f8_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev8)
+        f8_tf = w.fwd_flops() / (f8_ms * 1e-3) / 1e12
+        # half the flops (S = Q K^T) at the e4m3 rate (2x bf16, the nominal ratio), half at bf16
+        mixed_peak = peak / 0.75
+        rows[f"{w.name}_fp8_fwd"] = {"ms": round(f8_ms, 4), "TFLOP/s": round(f8_tf, 1),
+                                     "frac_of_peak": round(f8_tf / mixed_peak, 3),
+                                     "peak": round(mixed_peak, 1),
+                                     "note": "e4m3 Q, K; bf16 V, O; 4*B*H*N^2*D flops; peak = measured bf16 "
+                                             "burst / 0.75 (S at 2x the bf16 rate, P V at bf16)"}
+        del q8, k8, v8, o8, l8
 
     # ---- extra memory versus a materialised-scores attention (arithmetic)
     naive_scores = w.B * w.H * w.Nq * w.Nk * 4
