@@ -75,6 +75,7 @@ struct FwdBarriers {
     uint64_t full[8];
     uint64_t empty[8];
     uint64_t s_full[2];
+    uint64_t p_half[2];   // P columns 0..63 of tile t are in TMEM
     uint64_t p_ready[2];
     uint64_t o_final;
     uint64_t merge_ready;
@@ -140,6 +141,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(&bars->s_full[t], 1);
+            mbar_init(&bars->p_half[t], 128);
             mbar_init(&bars->p_ready[t], 128);
         }
         mbar_init(&bars->o_final, 1);
@@ -238,21 +240,34 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // descriptor's leading-byte offset (rank 0 and non-cluster launches
             // were correct).  The single N = D instruction is kept otherwise.
             const bool pv_by_block = (D > 64) && (nranks > 1);
-            auto issue_pv = [&](unsigned tO, unsigned tS, uint32_t v_off, unsigned acc0) {
+            // P V over the keys [16 kk0, 16 kk1) of the tile (K steps kk0..kk1-1)
+            auto issue_pv = [&](unsigned tO, unsigned tS, uint32_t v_off, unsigned acc0, int kk0, int kk1) {
                 if (pv_by_block) {
                     constexpr unsigned idesc_o64 = make_idesc_bf16(128, 64, 0, 1);
 #pragma unroll
                     for (int blk = 0; blk < D / 64; ++blk)
 #pragma unroll
-                        for (int kk = 0; kk < kTileN / 16; ++kk)
+                        for (int kk = kk0; kk < kk1; ++kk)
                             mma_ts_lo(tO + 64 * blk, tS + kk * 8,
                                       ring_v_lo + v_off + blk * (Cfg::kBoxBytes >> 4) + mnmajor_step(kk), idesc_o64,
                                       (acc0 | kk) ? 1u : 0u);
                 } else {
 #pragma unroll
-                    for (int kk = 0; kk < kTileN / 16; ++kk)
+                    for (int kk = kk0; kk < kk1; ++kk)
                         mma_ts_lo(tO, tS + kk * 8, ring_v_lo + v_off + mnmajor_step(kk), idesc_o, (acc0 | kk) ? 1u : 0u);
                 }
+            };
+            // P V in two halves: the first four K steps as soon as the softmax has
+            // stored P's first 64 columns, the rest once the whole P is in TMEM
+            auto pv_halves = [&](int t, unsigned parity, uint32_t v_off, unsigned acc0) -> bool {
+                const unsigned tO = t ? tO1 : tO0, tS = t ? tS1 : tS0;
+                if (!mbar_wait(&bars->p_half[t], parity, abort_flag)) return false;
+                tc_fence_after();
+                issue_pv(tO, tS, v_off, acc0, 0, kTileN / 32);
+                if (!mbar_wait(&bars->p_ready[t], parity, abort_flag)) return false;
+                tc_fence_after();
+                issue_pv(tO, tS, v_off, acc0, kTileN / 32, kTileN / 16);
+                return true;
             };
             uint32_t k_off = 0;
             int k_stage = 0;
@@ -275,9 +290,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int j = 0; ok && j < n_kv; ++j) {
                     const int t = j & 1;
                     const int i = j >> 1;  // iteration of slot t
-                    if (!(ok = mbar_wait(&bars->p_ready[t], i & 1, abort_flag))) break;
-                    tc_fence_after();
-                    issue_pv(t ? tO1 : tO0, t ? tS1 : tS0, v_off[t], i > 0 ? 1u : 0u);
+                    if (!(ok = pv_halves(t, i & 1, v_off[t], i > 0 ? 1u : 0u))) break;
                     mma_commit(&bars->empty[v_stage[t]]);
                     if (j + 2 < n_kv) {
                         if (!(ok = next_tile(k_off, k_stage))) break;
@@ -305,9 +318,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 int v_stage = 0;
                 if (!(ok = next_tile(v_off, v_stage))) break;
                 // tile 0: O_0 += P_0 V_j, then S_0 = Q_0 K_{j+1}^T
-                if (!(ok = mbar_wait(&bars->p_ready[0], j & 1, abort_flag))) break;
-                tc_fence_after();
-                issue_pv(tO0, tS0, v_off, acc0);
+                if (!(ok = pv_halves(0, j & 1, v_off, acc0))) break;
                 if (more) {
                     if (!(ok = next_tile(k_off, k_stage))) break;
                     tc_fence_after();
@@ -315,9 +326,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     mma_commit(&bars->s_full[0]);
                 }
                 // tile 1: O_1 += P_1 V_j, then S_1 = Q_1 K_{j+1}^T
-                if (!(ok = mbar_wait(&bars->p_ready[1], j & 1, abort_flag))) break;
-                tc_fence_after();
-                issue_pv(tO1, tS1, v_off, acc0);
+                if (!(ok = pv_halves(1, j & 1, v_off, acc0))) break;
                 mma_commit(&bars->empty[v_stage]);
                 if (more) {
                     issue_s(tS1, q_lo1, k_off);
@@ -354,6 +363,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!live) {
             for (int i = 0; i < n_mine; ++i) {
                 if (!(ok = mbar_wait(&bars->s_full[t], i & 1, abort_flag))) break;
+                mbar_arrive(&bars->p_half[t]);
                 mbar_arrive(&bars->p_ready[t]);
             }
         } else {
@@ -416,11 +426,20 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         pk[c / 2] = pack_bf16x2(p0, p1);
                     }
                     tmem_st16(tS + c0 / 2, pk);
+                    if (c0 == kTileN / 2 - 32 && !rescale) {
+                        // P's first 64 columns are in TMEM and O needs no rescale:
+                        // their P V steps may start
+                        tmem_wait_st();
+                        tc_fence_before();
+                        mbar_arrive(&bars->p_half[t]);
+                    }
                 }
                 l += ((rsa[0] + rsa[1]) + (rsa[2] + rsa[3])) + ((rsa[4] + rsa[5]) + (rsa[6] + rsa[7]));
                 if (rescale) {
-                    // PV_t(j-1) has completed (it was issued before S_t(j), whose
-                    // commit we waited on), so O_t can be rescaled in place.
+                    // PV_t of the previous key tile has completed (it was issued before
+                    // S_t of this one, whose commit we waited on), so O_t can be rescaled
+                    // in place; this warp's first-half signal waits for it, and P V
+                    // starts only when all four warps have signalled
 #pragma unroll
                     for (int c0 = 0; c0 < D; c0 += 32) {
                         uint32_t ov[32];
@@ -433,6 +452,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 tmem_wait_st();
                 tc_fence_before();
+                if (rescale) mbar_arrive(&bars->p_half[t]);
                 mbar_arrive(&bars->p_ready[t]);
             }
         }
