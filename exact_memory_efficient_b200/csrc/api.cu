@@ -51,9 +51,9 @@ struct DeviceInfo {
     bool sm100 = false;
     int sm_count = 0;
     // clusters of the tensor-core forward (index 0: D = 64, 1: D = 128,
-    // 2: D = 128 with e4m3 Q/K) that can be resident at once, per cluster
-    // size; -1 until first queried
-    int fwd_clusters[3][17];
+    // 2: D = 128 with e4m3 Q/K; +3 for the single-query-tile instantiations)
+    // that can be resident at once, per cluster size; -1 until first queried
+    int fwd_clusters[6][17];
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -97,10 +97,11 @@ mea_status_t device_info(DeviceInfo** out) {
 
 // Clusters of `size` CTAs of the bf16 forward that fit on the device at once
 // (cached; 0 if the query fails, which only disables that cluster size).
-int fwd_max_clusters(DeviceInfo* d, int D, bool fp8, int size) {
+int fwd_max_clusters(DeviceInfo* d, int D, bool fp8, int Nq, int size) {
     std::lock_guard<std::mutex> lk(g_mu);
-    int& n = d->fwd_clusters[fp8 ? 2 : (D == 128 ? 1 : 0)][size];
-    if (n < 0) n = mea::fwd_bf16_max_active_clusters(D, fp8, size);
+    const int single = (D == 128 && Nq <= 128) ? 3 : 0;   // the kernel's deep-ring instantiation
+    int& n = d->fwd_clusters[(fp8 ? 2 : (D == 128 ? 1 : 0)) + single][size];
+    if (n < 0) n = mea::fwd_bf16_max_active_clusters(D, fp8, Nq, size);
     return n;
 }
 
@@ -196,7 +197,7 @@ mea_status_t tc_forward(const void* q, const void* k, const void* v, void* o, fl
         if (base * 2 <= dev->sm_count) {
             long long best = base;
             for (int c = 2; c <= 16 && key_tiles >= 2 * c; ++c) {
-                if (base > fwd_max_clusters(dev, D, fp8, c)) continue;
+                if (base > fwd_max_clusters(dev, D, fp8, Nq, c)) continue;
                 if (base * c > best) {
                     best = base * c;
                     chunks = c;

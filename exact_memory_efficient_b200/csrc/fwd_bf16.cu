@@ -55,8 +55,11 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
 
 // F8: Q and K are e4m3 (one byte per element) and S = Q K^T runs as
-// kind::f8f6f4; V, P and O stay bf16.
-template <int D, bool F8 = false>
+// kind::f8f6f4; V, P and O stay bf16.  DEEP: one more ring stage (the
+// launches whose CTAs all hold a single query tile, i.e. decode, stream K/V
+// with little compute per byte and gain from the deeper prefetch; two-tile
+// launches do not).
+template <int D, bool F8 = false, bool DEEP = false>
 struct FwdCfg {
     static constexpr int kQKElem = F8 ? 1 : 2;                // bytes per Q/K element
     static constexpr int kQKBox = 128 / kQKElem;              // Q/K elements per 128-byte box row
@@ -64,7 +67,7 @@ struct FwdCfg {
     static constexpr int kVBytes = kTileN * D * 2;            // one V tile
     static constexpr int kTileBytes = kVBytes;                // one ring stage (a K tile uses its start)
     static constexpr int kQBytes = kTileM * D * kQKElem;      // one Q tile
-    static constexpr int kStages = F8 ? ((D == 128) ? 5 : 7) : ((D == 128) ? 4 : 6);
+    static constexpr int kStages = (F8 ? ((D == 128) ? 5 : 7) : ((D == 128) ? 4 : 6)) + (DEEP ? 1 : 0);
     static constexpr int kBoxBytes = 128 * 128;               // one 128-byte-wide box of 128 rows
     static constexpr int kSmemData = 2 * kQBytes + kStages * kTileBytes;
     static constexpr int kSmemBytes = kSmemData + 1024 /*barriers*/ + 1024 /*alignment slack*/;
@@ -72,7 +75,7 @@ struct FwdCfg {
 
 struct FwdBarriers {
     uint64_t q_full;
-    uint64_t full[8];
+    uint64_t full[8];    // ring stages (at most 8)
     uint64_t empty[8];
     uint64_t s_full[2];
     uint64_t p_half[2];   // P columns 0..63 of tile t are in TMEM
@@ -97,18 +100,21 @@ __device__ __forceinline__ float* part_ml(uint8_t* smem, int t, int r) {
 }
 static_assert(2 * 128 * (128 + 4) * 4 + 2 * 128 * 2 * 4 <= FwdCfg<128>::kSmemData, "merge area (D=128)");
 static_assert(2 * 128 * (128 + 4) * 4 + 2 * 128 * 2 * 4 <= FwdCfg<128, true>::kSmemData, "merge area (D=128, fp8)");
+static_assert(FwdCfg<128, true, true>::kStages <= 8 && FwdCfg<64, false, true>::kStages <= 8, "ring barriers");
+static_assert(FwdCfg<128, true, true>::kSmemBytes <= 227 * 1024 && FwdCfg<128, false, true>::kSmemBytes <= 227 * 1024,
+              "shared memory");
 static_assert(2 * 128 * (64 + 4) * 4 + 2 * 128 * 2 * 4 <= FwdCfg<64>::kSmemData, "merge area (D=64)");
 
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-template <int D, bool F8>
+template <int D, bool F8, bool DEEP>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ o,
                 float* __restrict__ lse, int Nq, int Nk, float scale, int chunk_len) {
-    using Cfg = FwdCfg<D, F8>;
+    using Cfg = FwdCfg<D, F8, DEEP>;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment of the shared-memory address (not of the generic
     // pointer: in a cluster launch each CTA's shared window can sit at a
@@ -598,10 +604,10 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
 }
 
-template <int D, bool F8>
+template <int D, bool F8, bool DEEP>
 cudaError_t launch_d(const Bf16FwdArgs& a, cudaStream_t stream) {
-    using Cfg = FwdCfg<D, F8>;
-    auto kern = fwd_bf16_kernel<D, F8>;
+    using Cfg = FwdCfg<D, F8, DEEP>;
+    auto kern = fwd_bf16_kernel<D, F8, DEEP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int q_tiles = (a.Nq + 2 * kTileM - 1) / (2 * kTileM);
@@ -629,10 +635,10 @@ cudaError_t launch_d(const Bf16FwdArgs& a, cudaStream_t stream) {
     return cudaLaunchKernelEx(&cfg, kern, a.tm_q, a.tm_k, a.tm_v, a.o, a.lse, a.Nq, a.Nk, a.scale, a.chunk_len);
 }
 
-template <int D, bool F8>
+template <int D, bool F8, bool DEEP>
 int max_active_clusters_d(int cluster) {
-    using Cfg = FwdCfg<D, F8>;
-    auto kern = fwd_bf16_kernel<D, F8>;
+    using Cfg = FwdCfg<D, F8, DEEP>;
+    auto kern = fwd_bf16_kernel<D, F8, DEEP>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
         return 0;
     if (cluster > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
@@ -658,18 +664,31 @@ int max_active_clusters_d(int cluster) {
 
 }  // namespace
 
-int fwd_bf16_max_active_clusters(int D, bool fp8_qk, int cluster) {
+// The deep-ring variant is used at D = 128 when every CTA holds a single query
+// tile (Nq <= 128).
+bool use_deep(int D, int Nq) { return D == 128 && Nq <= kTileM; }
+
+int fwd_bf16_max_active_clusters(int D, bool fp8_qk, int Nq, int cluster) {
     if (cluster < 1 || cluster > 16) return 0;
-    if (fp8_qk) return D == 128 ? max_active_clusters_d<128, true>(cluster) : 0;
-    if (D == 64) return max_active_clusters_d<64, false>(cluster);
-    if (D == 128) return max_active_clusters_d<128, false>(cluster);
+    const bool deep = use_deep(D, Nq);
+    if (fp8_qk) {
+        if (D != 128) return 0;
+        return deep ? max_active_clusters_d<128, true, true>(cluster) : max_active_clusters_d<128, true, false>(cluster);
+    }
+    if (D == 64) return max_active_clusters_d<64, false, false>(cluster);
+    if (D == 128)
+        return deep ? max_active_clusters_d<128, false, true>(cluster) : max_active_clusters_d<128, false, false>(cluster);
     return 0;
 }
 
 cudaError_t launch_fwd_bf16(const Bf16FwdArgs& a, cudaStream_t stream) {
-    if (a.fp8_qk) return a.D == 128 ? launch_d<128, true>(a, stream) : cudaErrorInvalidValue;
-    if (a.D == 64) return launch_d<64, false>(a, stream);
-    if (a.D == 128) return launch_d<128, false>(a, stream);
+    const bool deep = use_deep(a.D, a.Nq);
+    if (a.fp8_qk) {
+        if (a.D != 128) return cudaErrorInvalidValue;
+        return deep ? launch_d<128, true, true>(a, stream) : launch_d<128, true, false>(a, stream);
+    }
+    if (a.D == 64) return launch_d<64, false, false>(a, stream);
+    if (a.D == 128) return deep ? launch_d<128, false, true>(a, stream) : launch_d<128, false, false>(a, stream);
     return cudaErrorInvalidValue;
 }
 

@@ -57,9 +57,10 @@ struct Bf16FwdArgs {
     bool fp8_qk = false;  // q, k are e4m3 (maps of uint8, box {128, 128, 1}); D = 128 only
 };
 cudaError_t launch_fwd_bf16(const Bf16FwdArgs& a, cudaStream_t stream);
-// Clusters of `cluster` CTAs of the bf16 forward for head dim D that can be
-// resident at once (cudaOccupancyMaxActiveClusters); 0 on failure.
-int fwd_bf16_max_active_clusters(int D, bool fp8_qk, int cluster);
+// Clusters of `cluster` CTAs of the tensor-core forward instantiation that a
+// launch with these D, operand type and Nq uses that can be resident at once
+// (cudaOccupancyMaxActiveClusters); 0 on failure.
+int fwd_bf16_max_active_clusters(int D, bool fp8_qk, int Nq, int cluster);
 
 // bf16 backward (bwd_bf16.cu).
 struct Bf16BwdArgs {
