@@ -55,10 +55,10 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
 
 // F8: Q and K are e4m3 (one byte per element) and S = Q K^T runs as
-// kind::f8f6f4; V, P and O stay bf16.  DEEP: one more ring stage (the
-// launches whose CTAs all hold a single query tile, i.e. decode, stream K/V
-// with little compute per byte and gain from the deeper prefetch; two-tile
-// launches do not).
+// kind::f8f6f4; V, P and O stay bf16.  DEEP: for launches whose CTAs all hold
+// a single query tile (decode): one Q buffer, and the space of the second one
+// plus the rest of shared memory goes to the K/V ring (such launches stream
+// K/V with little compute per byte and gain from the deeper prefetch).
 template <int D, bool F8 = false, bool DEEP = false>
 struct FwdCfg {
     static constexpr int kQKElem = F8 ? 1 : 2;                // bytes per Q/K element
@@ -67,9 +67,10 @@ struct FwdCfg {
     static constexpr int kVBytes = kTileN * D * 2;            // one V tile
     static constexpr int kTileBytes = kVBytes;                // one ring stage (a K tile uses its start)
     static constexpr int kQBytes = kTileM * D * kQKElem;      // one Q tile
-    static constexpr int kStages = (F8 ? ((D == 128) ? 5 : 7) : ((D == 128) ? 4 : 6)) + (DEEP ? 1 : 0);
+    static constexpr int kQTiles = DEEP ? 1 : 2;                // Q buffers
+    static constexpr int kStages = DEEP ? 6 : (F8 ? ((D == 128) ? 5 : 7) : ((D == 128) ? 4 : 6));
     static constexpr int kBoxBytes = 128 * 128;               // one 128-byte-wide box of 128 rows
-    static constexpr int kSmemData = 2 * kQBytes + kStages * kTileBytes;
+    static constexpr int kSmemData = kQTiles * kQBytes + kStages * kTileBytes;
     static constexpr int kSmemBytes = kSmemData + 1024 /*barriers*/ + 1024 /*alignment slack*/;
 };
 
@@ -121,7 +122,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // different generic offset) for the 128-byte-swizzle atoms
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* sQ = smem;                               // Q_0 then Q_1
-    uint8_t* sRing = smem + 2 * Cfg::kQBytes;         // kStages tiles
+    uint8_t* sRing = smem + Cfg::kQTiles * Cfg::kQBytes;   // kStages tiles
     FwdBarriers* bars = reinterpret_cast<FwdBarriers*>(smem + Cfg::kSmemData);
 
     const unsigned warp = warp_id();
@@ -134,7 +135,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int m0 = (blockIdx.x / nranks) * (2 * kTileM);
     // A CTA whose rows all fall in its first query tile (decode-shaped calls,
     // the last tile pair of a ragged Nq) issues no work for the second tile.
-    const bool two = (m0 + kTileM) < Nq;
+    const bool two = !DEEP && (m0 + kTileM) < Nq;   // DEEP launches have Nq <= 128
     const int c_begin = (nranks > 1) ? (int)rank * chunk_len : 0;
     const int c_end = (nranks > 1) ? min(Nk, c_begin + chunk_len) : Nk;
     const int n_kv = (c_end > c_begin) ? (c_end - c_begin + kTileN - 1) / kTileN : 0;
