@@ -104,6 +104,11 @@ fwd_f32_kernel(const float* __restrict__ q, const float* __restrict__ k, const f
 
         for (int j0 = c_begin + 32 * kg; j0 < c_end; j0 += 32 * warps_per_row) {
             const int nvalid = min(32, c_end - j0);
+            // Value rows do not depend on the scores: for D <= 64 (DPL <= 2) they
+            // are loaded together with the key rows, so both streams are in flight
+            // at once (this loop is bound by memory latency, not arithmetic).
+            constexpr bool kVEarly = DPL <= 2;
+            float vbuf[kVEarly ? 32 : 1][DPL];
             // scores of the 32 keys of this group, reduce-scattered to lane j
             float pd[32];
 #pragma unroll
@@ -111,9 +116,14 @@ fwd_f32_kernel(const float* __restrict__ q, const float* __restrict__ k, const f
                 float kv[DPL];
                 if (j < nvalid) {
                     load_dims<DPL>(kh + (size_t)(j0 + j) * D + DPL * lane, kv);
+                    if constexpr (kVEarly) load_dims<DPL>(vh + (size_t)(j0 + j) * D + DPL * lane, vbuf[j]);
                 } else {
 #pragma unroll
                     for (int i = 0; i < DPL; ++i) kv[i] = 0.f;
+                    if constexpr (kVEarly) {
+#pragma unroll
+                        for (int i = 0; i < DPL; ++i) vbuf[j][i] = 0.f;
+                    }
                 }
                 float t = 0.f;
 #pragma unroll
@@ -130,14 +140,23 @@ fwd_f32_kernel(const float* __restrict__ q, const float* __restrict__ k, const f
 #pragma unroll
             for (int i = 0; i < DPL; ++i) st.acc[i] *= alpha;
             st.m = m_new;
-#pragma unroll 8
-            for (int j = 0; j < 32; ++j) {
-                const float pj = __shfl_sync(0xffffffffu, p, j);
-                if (j < nvalid) {
-                    float vv[DPL];
-                    load_dims<DPL>(vh + (size_t)(j0 + j) * D + DPL * lane, vv);
+            if constexpr (kVEarly) {
 #pragma unroll
-                    for (int i = 0; i < DPL; ++i) st.acc[i] = fmaf(pj, vv[i], st.acc[i]);
+                for (int j = 0; j < 32; ++j) {
+                    const float pj = __shfl_sync(0xffffffffu, p, j);   // 0 past nvalid
+#pragma unroll
+                    for (int i = 0; i < DPL; ++i) st.acc[i] = fmaf(pj, vbuf[j][i], st.acc[i]);
+                }
+            } else {
+#pragma unroll 8
+                for (int j = 0; j < 32; ++j) {
+                    const float pj = __shfl_sync(0xffffffffu, p, j);
+                    if (j < nvalid) {
+                        float vv[DPL];
+                        load_dims<DPL>(vh + (size_t)(j0 + j) * D + DPL * lane, vv);
+#pragma unroll
+                        for (int i = 0; i < DPL; ++i) st.acc[i] = fmaf(pj, vv[i], st.acc[i]);
+                    }
                 }
             }
         }
