@@ -274,7 +274,8 @@ mea_status_t mea_attn_fwd(const void* q, const void* k, const void* v, void* o, 
         if (Nq >= 8) { a.rows_per_cta = 8; a.warps_per_row = 1; }
         else if (Nq >= 4) { a.rows_per_cta = 4; a.warps_per_row = 2; }
         else if (Nq >= 2) { a.rows_per_cta = 2; a.warps_per_row = 4; }
-        else { a.rows_per_cta = 1; a.warps_per_row = 8; }
+        else { a.rows_per_cta = 1; a.warps_per_row = (D <= 64) ? 16 : 8; }   // 16 warps only within the
+                                                                            // D <= 64 register budget
         const long long base = (long long)BH * ((Nq + a.rows_per_cta - 1) / a.rows_per_cta);
         const long long target = 2LL * dev->sm_count;
         int chunks = 1;

@@ -65,14 +65,19 @@ struct alignas(16) Summary {
     float pad[2];
 };
 
+// Up to 16 warps per CTA for D <= 64 (a single query row then gets 16 warps of
+// key slices, for more loads in flight), 8 otherwise (register budget).
 template <int DPL>
-__global__ void __launch_bounds__(256)
+constexpr int kMaxWarps = (DPL <= 2) ? 16 : 8;
+
+template <int DPL>
+__global__ void __launch_bounds__(32 * kMaxWarps<DPL>)
 fwd_f32_kernel(const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
                float* __restrict__ o, float* __restrict__ lse,
                int Nq, int Nk, float scale, int rows_per_cta, int warps_per_row, int chunk_len) {
     constexpr int D = 32 * DPL;
-    __shared__ Summary<DPL> warp_sum_s[8];   // one per warp
-    __shared__ Summary<DPL> cta_sum_s[8];    // one per row of this CTA (read by cluster rank 0)
+    __shared__ Summary<DPL> warp_sum_s[kMaxWarps<DPL>];   // one per warp
+    __shared__ Summary<DPL> cta_sum_s[8];                 // one per row of this CTA (read by cluster rank 0)
 
     cg::cluster_group cluster = cg::this_cluster();
     const unsigned nranks = cluster.num_blocks();
