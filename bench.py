@@ -546,6 +546,23 @@ def run_ours(args):
     return 0
 
 
+def run_profile(name: str) -> int:
+    """Three forward (+ backward) calls of one workload through the public API, untimed."""
+    import exact_memory_efficient_b200 as m
+    w = make_workload(name)
+    torch.cuda.set_device(0)
+    q, k, v, do = (x.cuda() if x is not None else None for x in make_inputs(w, 0))
+    for _ in range(3):
+        o, lse = m.attention_forward(q, k, v, w.scale)
+        if do is not None:
+            m.attention_backward(q, k, v, o, lse, do, w.scale)
+    st = m.mea_last_device_error()
+    if st != m.MEA_OK:
+        raise RuntimeError(m.mea_status_string(st))
+    print(f"profile {name}: ok")
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -558,9 +575,14 @@ def main():
                          "headline workload, others are for profiling captures")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the end-to-end, fp32-row and CPU-baseline measurements (profiling captures)")
+    ap.add_argument("--profile", metavar="WORKLOAD", default=None,
+                    help="no timing: run this workload's forward (and backward, if it has one) three times and "
+                         "exit; the command profiling captures wrap")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.profile is not None:
+        return run_profile(args.profile)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
