@@ -13,22 +13,31 @@
 //   warp 0      TMEM allocator, then TMA producer (Q once, then K_0, V_0,
 //               K_1, V_1, ... ; no multicast)
 //   warp 1      MMA issuer (one thread): S_t = Q_t K_j^T into TMEM, then
-//               O_t += P_t V_j with P_t read from TMEM
-//   warps 2-5   softmax of query tile 0, warps 6-9 softmax of query tile 1
-//               (warp w reaches TMEM lanes 32*(w%4) .. 32*(w%4)+31):
-//               one thread per query row (TMEM lane), tcgen05.ld of S,
-//               exp2 with scale*log2(e) folded in, P written back to TMEM as
-//               bf16 over the S columns, O rescaled in TMEM when the reference
-//               maximum moves.
+//               O_t += P_t V_j with P_t read from TMEM, in two halves of
+//               64 keys (the first as soon as the softmax has stored it)
+//   warps 2-5   softmax of TMEM slot 0, warps 6-9 of slot 1 (warp w reaches
+//               TMEM lanes 32*(w%4) .. 32*(w%4)+31): one thread per query row
+//               (TMEM lane), tcgen05.ld of S, exp2 with scale*log2(e) folded
+//               in, P written back to TMEM as bf16 over the S columns, O
+//               rescaled in TMEM when the reference maximum moves.
 // TMEM (512 columns): S_0 [0,128)  S_1 [128,256)  O_0 [256,256+D)  O_1 [384,384+D).
+// With two live query tiles slot t holds query tile t.  A CTA whose rows all
+// fit in its first tile (decode, or the last pair of a ragged Nq) runs both
+// slots on that tile over alternate key tiles and merges the two summaries at
+// the end, so one slot's softmax still overlaps the other's MMAs.
+//
+// Instantiations: F8 takes e4m3 Q and K (S on kind::f8f6f4; V, P, O bf16);
+// DEEP (launches with Nq <= 128 at D = 128) keeps one Q buffer and gives the
+// rest of shared memory to a six-stage K/V ring.
 //
 // Key split (decode-shaped calls): when a grid would leave most SMs idle (few
 // query tiles x heads), the keys of each (batch, head, query tile) are split
 // over the CTAs of a thread-block cluster.  Each CTA runs the recurrence over
 // its chunk and leaves the chunk summary of every row -- its reference maximum,
-// exp-sum and unnormalised accumulator -- in its shared memory; the cluster's
-// first CTA merges the summaries through distributed shared memory with the
-// two-block formulas and writes O and lse.  No global scratch is used.
+// exp-sum and unnormalised accumulator -- in its shared memory; the CTAs then
+// merge the summaries through distributed shared memory with the two-block
+// formulas, each writing a slice of the head dims of O (and the first, lse).
+// No global scratch is used.
 //
 // Reference maximum: a row's exponentials are taken relative to a reference
 // value m_ref that is raised to the true running maximum only when the new
