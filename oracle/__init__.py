@@ -24,5 +24,6 @@ from .attention import (  # noqa: F401
     attention_backward_rows,
     attention_backward_keys,
     chunked_forward_2d,
+    combine_partials,
     combine_two_blocks,
 )

@@ -217,6 +217,26 @@ def combine_two_blocks(m1, l1, acc1, m2, l2, acc2):
     return m, l1 * a1 + l2 * a2, acc1 * a1[..., None] + acc2 * a2[..., None]
 
 
+def combine_partials(o_parts, lse_parts):
+    """Merge R results computed over disjoint key ranges into the result over all of them.
+
+    Each part r is exact attention over its own keys: O_r = sum_j p_rj v_j / l_r
+    with lse_r = ln l_r (in the scaled-score units of lse).  The chunk summary
+    of "Self-attention Does Not Need O(n^2) Memory" (English summary, the bullet
+    on summarising chunk results) is (m_r, l_r, acc_r) with acc_r = l_r O_r e^{m_r};
+    merged with the two-block formulas of "当注意力成为瓶颈" (section IO感知)
+    it gives   lse = ln sum_r e^{lse_r},   O = sum_r e^{lse_r - lse} O_r.
+    o_parts [R, ..., D], lse_parts [R, ...] -> (O [..., D], lse [...]).
+    """
+    o_parts, lse_parts = _f64(o_parts), _f64(lse_parts)
+    m = lse_parts.max(axis=0)
+    w = np.exp(lse_parts - m)
+    total = w.sum(axis=0)
+    lse = m + np.log(total)
+    o = (w[..., None] * o_parts).sum(axis=0) / total[..., None]
+    return o, lse
+
+
 def chunked_forward_2d(q, k, v, scale, block):
     """The method's own order: keys/values in blocks, each block summarised as
     (running max m, total weight l, weighted value sum acc), summaries merged,

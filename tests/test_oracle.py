@@ -406,3 +406,36 @@ def test_gqa_single_group_is_mha():
     b = oracle.attention_backward(q, k, v, do, 0.5)
     for x, y in zip(a, b):
         np.testing.assert_allclose(x, y, atol=1e-14)
+
+
+# ------------------------------------------------ merging key-range results
+
+@pytest.mark.parametrize("R", [1, 2, 3, 7])
+def test_combine_partials_reaches_the_full_result(R):
+    """Attention over R disjoint key ranges, merged, equals attention over all keys (any split)."""
+    rng = np.random.default_rng(R)
+    q = rng.standard_normal((5, 8))
+    k = rng.standard_normal((40, 8)) * 2.0
+    v = rng.standard_normal((40, 8))
+    cuts = np.sort(rng.choice(np.arange(1, 40), R - 1, replace=False)) if R > 1 else np.array([], dtype=int)
+    bounds = np.concatenate([[0], cuts, [40]])
+    parts = [oracle.attention_forward_2d(q, k[a:b], v[a:b], 0.7) for a, b in zip(bounds[:-1], bounds[1:])]
+    o, lse = oracle.combine_partials(np.stack([p_[0] for p_ in parts]), np.stack([p_[1] for p_ in parts]))
+    ro, rl = oracle.attention_forward_2d(q, k, v, 0.7)
+    np.testing.assert_allclose(o, ro, atol=1e-13)
+    np.testing.assert_allclose(lse, rl, atol=1e-13)
+
+
+def test_combine_partials_closed_form():
+    """Two parts with lse ln 1 and ln 3: weights 1/4 and 3/4, lse ln 4."""
+    o, lse = oracle.combine_partials(np.array([[[2.0, 0.0]], [[6.0, 4.0]]]), np.array([[0.0], [np.log(3.0)]]))
+    np.testing.assert_allclose(o, [[0.25 * 2 + 0.75 * 6, 0.75 * 4]], atol=1e-15)
+    np.testing.assert_allclose(lse, [np.log(4.0)], atol=1e-15)
+
+
+def test_combine_partials_large_lse_is_finite():
+    """Parts whose lse are ~1e3 apart: the merge is taken relative to the largest lse."""
+    o, lse = oracle.combine_partials(np.array([[[1.0]], [[3.0]]]), np.array([[1000.0], [-5.0]]))
+    assert np.isfinite(o).all() and np.isfinite(lse).all()
+    np.testing.assert_allclose(o, [[1.0]], atol=1e-15)
+    np.testing.assert_allclose(lse, [1000.0], atol=1e-12)
