@@ -29,7 +29,7 @@ __all__ = [
     "MEA_BWD_ALL", "MEA_BWD_PREPROCESS", "MEA_BWD_MAIN", "MEA_BWD_FINALIZE",
     "mea_attn_fwd", "mea_attn_bwd", "mea_attn_bwd_phase", "mea_attn_bwd_workspace_size", "mea_attn_bwd_noalloc",
     "mea_attn_fwd_gqa", "mea_attn_bwd_gqa", "mea_attn_bwd_gqa_workspace_size", "mea_attn_fwd_fp8",
-    "mea_last_device_error",
+    "mea_attn_combine", "mea_last_device_error",
     "mea_selftest_bounded_wait", "mea_status_string", "mea_last_error_message", "mea_version", "attention_forward", "attention_backward",
 ]
 
@@ -95,6 +95,8 @@ def load_library() -> ctypes.CDLL:
     lib.mea_attn_bwd_gqa.restype = i
     lib.mea_attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, f, vp]
     lib.mea_attn_fwd_fp8.restype = i
+    lib.mea_attn_combine.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i, vp, vp, i, i, i, i, i, vp]
+    lib.mea_attn_combine.restype = i
     lib.mea_selftest_bounded_wait.argtypes = [vp, vp]
     lib.mea_selftest_bounded_wait.restype = i
     lib.mea_last_device_error.argtypes = [vp]
@@ -273,6 +275,28 @@ def mea_attn_fwd_fp8(q, k, v, o, lse, scale: float, q_descale: float, k_descale:
     st = load_library().mea_attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Nq, Nk, D,
                                           float(scale), float(q_descale), float(k_descale), _stream_handle(stream))
     _check(st, "mea_attn_fwd_fp8")
+
+
+def mea_attn_combine(o_parts, lse_parts, o, lse, stream=None) -> None:
+    """C ``mea_attn_combine``: merge results over disjoint key ranges.  ``o_parts`` and
+    ``lse_parts`` are sequences of R CUDA tensors shaped like ``o`` [B,H,Nq,D] and ``lse``
+    [B,H,Nq] (fp32); writes the merged o and lse."""
+    B, H, Nq, D = _bhnd(o, "o")
+    R = len(o_parts)
+    if R != len(lse_parts) or R < 1:
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_combine: one lse part per o part")
+    for op, lp in zip(o_parts, lse_parts):
+        if tuple(op.shape) != tuple(o.shape) or op.dtype != o.dtype or not op.is_contiguous():
+            raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_combine: o parts must match o")
+        if tuple(lp.shape) != (B, H, Nq) or lp.dtype != torch.float32 or not lp.is_contiguous():
+            raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_combine: lse parts must be fp32 [B, H, Nq]")
+    if tuple(lse.shape) != (B, H, Nq) or lse.dtype != torch.float32:
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_combine: lse must be fp32 [B, H, Nq]")
+    optr = (ctypes.c_void_p * R)(*[_ptr(t) for t in o_parts])
+    lptr = (ctypes.c_void_p * R)(*[_ptr(t) for t in lse_parts])
+    st = load_library().mea_attn_combine(optr, lptr, R, _ptr(o), _ptr(lse), B, H, Nq, D, _dtype_code(o),
+                                          _stream_handle(stream))
+    _check(st, "mea_attn_combine")
 
 
 def mea_selftest_bounded_wait(gave_up, stream=None) -> None:

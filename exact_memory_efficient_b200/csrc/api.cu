@@ -458,6 +458,41 @@ mea_status_t mea_attn_fwd_fp8(const void* q, const void* k, const void* v, void*
     return tc_forward(q, k, v, o, lse, B * H_kv, rows, Nk, D, eff, true, dev, static_cast<cudaStream_t>(stream));
 }
 
+mea_status_t mea_attn_combine(const void* const* o_parts, const float* const* lse_parts, int R, void* o,
+                              float* lse, int B, int H, int Nq, int D, mea_dtype_t dtype, void* stream) {
+    if (dtype != MEA_DTYPE_F32 && dtype != MEA_DTYPE_BF16) return MEA_ERR_INVALID_ARG;
+    if (R < 1 || R > mea::kCombineMaxParts)
+        return fail(MEA_ERR_UNSUPPORTED, "mea_attn_combine", "1 to 16 parts");
+    if (B < 0 || H < 0 || Nq < 0 || D <= 0) return MEA_ERR_INVALID_ARG;
+    if (D % 8 != 0 || D > 256) return fail(MEA_ERR_UNSUPPORTED, "mea_attn_combine", "D a multiple of 8, at most 256");
+    const long long rows = (long long)B * H * Nq;
+    if (rows * D >= (1LL << 40)) return MEA_ERR_INVALID_ARG;
+    if (rows == 0) return MEA_OK;
+    if (!o_parts || !lse_parts || !o || !lse) return MEA_ERR_INVALID_ARG;
+    mea::CombineArgs a;
+    for (int r = 0; r < R; ++r) {
+        if (!o_parts[r] || !lse_parts[r]) return MEA_ERR_INVALID_ARG;
+        if (!aligned16(o_parts[r]) || !aligned4(lse_parts[r])) return MEA_ERR_MISALIGNED;
+        a.o_parts[r] = o_parts[r];
+        a.lse_parts[r] = lse_parts[r];
+    }
+    for (int r = R; r < mea::kCombineMaxParts; ++r) {
+        a.o_parts[r] = nullptr;
+        a.lse_parts[r] = nullptr;
+    }
+    if (!aligned16(o) || !aligned4(lse)) return MEA_ERR_MISALIGNED;
+    a.o = o;
+    a.lse = lse;
+    a.rows = rows;
+    a.D = D;
+    a.R = R;
+    DeviceInfo* dev = nullptr;
+    mea_status_t st = device_info(&dev);
+    if (st != MEA_OK) return st;
+    return cuda_status(mea::launch_combine(a, dtype == MEA_DTYPE_BF16, static_cast<cudaStream_t>(stream)),
+                       "combine launch");
+}
+
 mea_status_t mea_attn_bwd_gqa_workspace_size(int B, int H, int H_kv, int Nq, int Nk, int D, mea_dtype_t dtype,
                                              size_t* bytes) {
     int rows = 0;

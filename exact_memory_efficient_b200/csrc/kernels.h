@@ -25,7 +25,21 @@ struct F32FwdArgs {
 };
 cudaError_t launch_fwd_f32(const F32FwdArgs& a, cudaStream_t stream);
 
-// fp32 SIMT backward (bwd_f32.cu).  Row term D_i in `delta` (workspace).
+// Merge of results over disjoint key ranges (combine.cu).  Pointer arrays are
+// passed by value; every part and the output are [rows, D] with rows = B*H*Nq.
+constexpr int kCombineMaxParts = 16;
+struct CombineArgs {
+    const void* o_parts[kCombineMaxParts];
+    const float* lse_parts[kCombineMaxParts];
+    void* o;
+    float* lse;
+    long long rows;
+    int D;
+    int R;
+};
+cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t stream);
+
+// fp32 SIMT backward (bwd_f32.cu).// fp32 SIMT backward (bwd_f32.cu).  Row term D_i in `delta` (workspace).
 struct F32BwdArgs {
     const float* q;
     const float* k;

@@ -221,6 +221,33 @@ mea_status_t mea_attn_fwd_fp8(const void* q, const void* k, const void* v,
                               float q_descale, float k_descale, void* stream);
 
 /*
+ * Merge of results computed over disjoint key ranges (key / sequence split).
+ *
+ * Source: "Self-attention Does Not Need O(n^2) Memory" (English summary, the
+ * bullet on summarising the results of key/value chunks) with the two-block
+ * formulas of "当注意力成为瓶颈从on困境到线性复杂度的技术突围" (section IO感知).
+ * Part r is mea_attn_fwd's output (o_r, lse_r) over the r-th key range; the
+ * merge gives exactly the attention over all keys:
+ *     lse = ln sum_r exp(lse_r),     o = sum_r exp(lse_r - lse) o_r.
+ * A part with lse = -inf (no keys) contributes nothing.
+ *
+ * o_parts, lse_parts: HOST arrays of R device pointers (1 <= R <= 16); each
+ * o part is [B, H, Nq, D] in `dtype`, each lse part [B, H, Nq] fp32.  The
+ * pointers may address memory of other GPUs that this one can read (peer
+ * access), so the merge can read remote parts directly.  o, lse: outputs of
+ * the same shapes.  Pointers 16-byte (o) / 4-byte (lse) aligned; D a multiple
+ * of 8, at most 256.  The backward of a key split needs no entry point of its
+ * own: each range runs mea_attn_bwd_phase with the merged o and lse, the fp32
+ * dQ accumulators of the ranges are summed between MAIN and FINALIZE, and dk,
+ * dv stay with their range.
+ * Errors: MEA_ERR_INVALID_ARG, MEA_ERR_UNSUPPORTED (R, D), MEA_ERR_MISALIGNED,
+ * MEA_ERR_CUDA.
+ */
+mea_status_t mea_attn_combine(const void* const* o_parts, const float* const* lse_parts, int R,
+                              void* o, float* lse, int B, int H, int Nq, int D,
+                              mea_dtype_t dtype, void* stream);
+
+/*
  * Backward pass that allocates nothing and takes no workspace.  The paper has
  * no counterpart: this is a deployment convenience of this library.
  *

@@ -183,3 +183,22 @@ def test_fp8_argument_validation(lib):
     assert fwd8(q=None) == 1
     assert fwd8(q=A + 8) == 3
     assert fwd8(Nq=0) == 0                 # no rows: no-op
+
+
+def test_combine_argument_validation(lib):
+    P = ctypes.c_void_p
+    def comb(R=2, D=64, dtype=BF16, optr=A, lptr=A, o=A, lse=A, Nq=16):
+        op = (P * max(R, 1))(*([optr] * max(R, 1)))
+        lp = (P * max(R, 1))(*([lptr] * max(R, 1)))
+        return lib.mea_attn_combine(op, lp, R, o, lse, 1, 2, Nq, D, dtype, None)
+
+    assert comb(R=0) == 2
+    assert comb(R=17) == 2
+    assert comb(D=60) == 2                 # D must be a multiple of 8
+    assert comb(D=264) == 2
+    assert comb(dtype=7) == 1
+    assert comb(optr=None) == 1
+    assert comb(optr=A + 8) == 3
+    assert comb(lptr=A + 2) == 3
+    assert comb(o=A + 4) == 3
+    assert comb(Nq=0) == 0                 # nothing to merge

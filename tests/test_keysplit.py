@@ -1,0 +1,159 @@
+"""Key (sequence) split: results over disjoint key ranges merged by mea_attn_combine (GPU).
+
+On one GPU the ranks of a key split are emulated as R key ranges processed one
+after another; every launch is an ordinary independent launch (nothing waits
+on another rank).  The all-gather of the parts is the list of R local buffers;
+the all-reduce of the backward's fp32 dQ accumulators is a sum over the R
+workspaces.  The oracle computes attention over all keys at once.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synthetic_inputs import custom, make_inputs, to_f64
+from tests._parity import BF16_GRAD, BF16_O, F32_O_MAX_ABS, assert_close, assert_lse_close, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def ranges(Nk, R, seed):
+    rng = np.random.default_rng(seed)
+    cuts = np.sort(rng.choice(np.arange(1, Nk), R - 1, replace=False)) if R > 1 else np.array([], dtype=int)
+    b = np.concatenate([[0], cuts, [Nk]])
+    return [(int(x), int(y)) for x, y in zip(b[:-1], b[1:])]
+
+
+def split_forward(qd, kd, vd, scale, rs):
+    import exact_memory_efficient_b200 as m
+    parts = [m.attention_forward(qd, kd[:, :, a:b].contiguous(), vd[:, :, a:b].contiguous(), scale) for a, b in rs]
+    o = torch.empty_like(qd)
+    lse = torch.empty(qd.shape[:3], dtype=torch.float32, device=qd.device)
+    m.mea_attn_combine([p[0] for p in parts], [p[1] for p in parts], o, lse)
+    return o, lse
+
+
+@pytest.mark.parametrize("dtype,R", [("bf16", 1), ("bf16", 2), ("bf16", 5), ("bf16", 16), ("f32", 3)])
+def test_combine_matches_oracle_merge(dtype, R):
+    """The merge alone, on random parts (lse spread over +-30 so the weights span many orders)."""
+    import exact_memory_efficient_b200 as m
+    g = torch.Generator().manual_seed(R)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    o_parts = [torch.randn(2, 3, 70, 64, generator=g).to(tdt) for _ in range(R)]
+    lse_parts = [(torch.rand(2, 3, 70, generator=g) * 60 - 30) for _ in range(R)]
+    o = torch.empty(2, 3, 70, 64, dtype=tdt, device="cuda")
+    lse = torch.empty(2, 3, 70, device="cuda")
+    m.mea_attn_combine([x.cuda() for x in o_parts], [x.cuda() for x in lse_parts], o, lse)
+    assert m.mea_last_device_error() == m.MEA_OK
+    ro, rl = oracle.combine_partials(np.stack([to_f64(x) for x in o_parts]), np.stack([to_f64(x) for x in lse_parts]))
+    tol = BF16_O if dtype == "bf16" else (F32_O_MAX_ABS, None)
+    assert_close(to_np(o), ro, *tol, what=f"combine {dtype} R={R}")
+    assert float(np.abs(to_np(lse) - rl).max()) <= 1e-5 * max(1.0, float(np.abs(rl).max()))
+
+
+def test_combine_skips_parts_without_keys():
+    """A part with lse = -inf (an empty key range) contributes nothing, even if its o holds NaN."""
+    import exact_memory_efficient_b200 as m
+    a = torch.randn(1, 1, 9, 64).to(torch.bfloat16).cuda()
+    nan = torch.full_like(a, float("nan"))
+    la = torch.randn(1, 1, 9).cuda()
+    ninf = torch.full_like(la, float("-inf"))
+    o = torch.empty_like(a)
+    lse = torch.empty_like(la)
+    m.mea_attn_combine([a, nan], [la, ninf], o, lse)
+    torch.cuda.synchronize()
+    assert torch.equal(o, a) and torch.allclose(lse, la)
+
+
+@pytest.mark.parametrize("B,H,Nq,Nk,D,R", [
+    (1, 2, 300, 1000, 128, 2),
+    (2, 3, 129, 777, 64, 3),
+    (1, 8, 1, 16384, 128, 8),     # decode: eight ranges of 2048 keys
+    (1, 4, 500, 4096, 128, 4),
+])
+def test_split_forward_bf16(B, H, Nq, Nk, D, R):
+    w = custom(B, H, Nq, Nk, D, "bf16", backward=False)
+    q, k, v, _ = make_inputs(w, 21)
+    o, lse = split_forward(q.cuda(), k.cuda(), v.cuda(), w.scale, ranges(Nk, R, 7))
+    ro, rl = oracle.attention_forward(to_f64(q), to_f64(k), to_f64(v), w.scale)
+    assert_close(to_np(o), ro, *BF16_O, what=f"split O {(B, H, Nq, Nk, D, R)}")
+    assert_lse_close(to_np(lse), rl, to_f64(q), to_f64(k), w.scale, what="split lse")
+
+
+def test_split_forward_f32():
+    w = custom(1, 4, 3, 6000, 64, "f32", backward=False)
+    q, k, v, _ = make_inputs(w, 22)
+    o, lse = split_forward(q.cuda(), k.cuda(), v.cuda(), w.scale, ranges(6000, 3, 8))
+    ro, rl = oracle.attention_forward(to_f64(q), to_f64(k), to_f64(v), w.scale)
+    assert_close(to_np(o), ro, F32_O_MAX_ABS, what="split fp32 O")
+    assert_lse_close(to_np(lse), rl, to_f64(q), to_f64(k), w.scale, what="split fp32 lse")
+
+
+@pytest.mark.parametrize("B,H,Nq,Nk,D,R", [(1, 2, 300, 1000, 128, 2), (1, 3, 257, 900, 64, 3)])
+def test_split_backward_bf16(B, H, Nq, Nk, D, R):
+    """Backward of a key split: each range recomputes P from the merged lse, the fp32 dQ
+    accumulators of the ranges are summed before the finalize phase, dk and dv stay local."""
+    import exact_memory_efficient_b200 as m
+    w = custom(B, H, Nq, Nk, D, "bf16")
+    q, k, v, do = make_inputs(w, 23)
+    qd, kd, vd, dod = (x.cuda() for x in (q, k, v, do))
+    rs = ranges(Nk, R, 9)
+    o, lse = split_forward(qd, kd, vd, w.scale, rs)
+    wsb = m.mea_attn_bwd_workspace_size(B, H, Nq, Nk, D)
+    acc_elems = B * H * Nq * D
+    dq = torch.empty_like(qd)
+    dks, dvs, wss = [], [], []
+    for a, b in rs:
+        ks, vs = kd[:, :, a:b].contiguous(), vd[:, :, a:b].contiguous()
+        dk, dv = torch.empty_like(ks), torch.empty_like(vs)
+        ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+        for ph in (m.MEA_BWD_PREPROCESS, m.MEA_BWD_MAIN):
+            m.mea_attn_bwd_phase(ph, qd, ks, vs, o, lse, dod, dq, dk, dv, w.scale, ws)
+        dks.append(dk)
+        dvs.append(dv)
+        wss.append(ws)
+    # the all-reduce of the dQ accumulators (fp32, at the start of each workspace)
+    acc0 = wss[0][:acc_elems * 4].view(torch.float32)
+    for ws in wss[1:]:
+        acc0 += ws[:acc_elems * 4].view(torch.float32)
+    m.mea_attn_bwd_phase(m.MEA_BWD_FINALIZE, qd, kd[:, :, rs[0][0]:rs[0][1]].contiguous(),
+                         vd[:, :, rs[0][0]:rs[0][1]].contiguous(), o, lse, dod, dq, dks[0], dvs[0], w.scale, wss[0])
+    assert m.mea_last_device_error() == m.MEA_OK
+    rq, rk, rv, _, _ = oracle.attention_backward(to_f64(q), to_f64(k), to_f64(v), to_f64(do), w.scale)
+    assert_close(to_np(dq), rq, *BF16_GRAD, what="split dQ", bf16_output=True)
+    assert_close(to_np(torch.cat(dks, dim=2)), rk, *BF16_GRAD, what="split dK", bf16_output=True)
+    assert_close(to_np(torch.cat(dvs, dim=2)), rv, *BF16_GRAD, what="split dV", bf16_output=True)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_keysplit_module_one_rank_nccl(dtype):
+    """The library's own key-split path (exact_memory_efficient_b200.keysplit with its CUDA ops)
+    in a one-rank NCCL group: the gather and all-reduce are trivial, every kernel and the
+    accumulator hand-off are the real ones."""
+    import socket
+    import torch.distributed as dist
+    from exact_memory_efficient_b200.keysplit import attention_backward_keysplit, attention_forward_keysplit
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            device_id=torch.device("cuda", 0))
+    try:
+        w = custom(1, 2, 200, 700, 64, dtype)
+        q, k, v, do = make_inputs(w, 24)
+        qd, kd, vd, dod = (x.cuda() for x in (q, k, v, do))
+        o, lse = attention_forward_keysplit(qd, kd, vd, w.scale)
+        dq, dk, dv = attention_backward_keysplit(qd, kd, vd, o, lse, dod, w.scale)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    rq, rk, rv, ro, rl = oracle.attention_backward(to_f64(q), to_f64(k), to_f64(v), to_f64(do), w.scale)
+    if dtype == "bf16":
+        assert_close(to_np(o), ro, *BF16_O, what="keysplit O")
+        for name, g_, r_ in (("dQ", dq, rq), ("dK", dk, rk), ("dV", dv, rv)):
+            assert_close(to_np(g_), r_, *BF16_GRAD, what=f"keysplit {name}", bf16_output=True)
+    else:
+        assert_close(to_np(o), ro, F32_O_MAX_ABS, what="keysplit fp32 O")
+        for name, g_, r_ in (("dQ", dq, rq), ("dK", dk, rk), ("dV", dv, rv)):
+            assert_close(to_np(g_), r_, F32_O_MAX_ABS, what=f"keysplit fp32 {name}")
