@@ -62,10 +62,12 @@ def source_sha(names=None) -> str:
     return h.hexdigest()[:16]
 
 
-# the files whose text decides each timed kernel's code
+# the files whose text decides each timed kernel's device code: its own source
+# and the device helpers it compiles (kernels.h holds host-side argument
+# structs and the other kernels' declarations)
 KERNEL_SOURCES = {
-    "bwd_main_kernel": ("bwd_bf16.cu", "ptx.cuh", "kernels.h"),
-    "fwd_bf16_kernel": ("fwd_bf16.cu", "ptx.cuh", "kernels.h"),
+    "bwd_main_kernel": ("bwd_bf16.cu", "ptx.cuh"),
+    "fwd_bf16_kernel": ("fwd_bf16.cu", "ptx.cuh"),
 }
 
 
@@ -483,6 +485,29 @@ def run_ours(args):
                                   "frac_of_peak": round(wg.bwd_flops() / (b_ms * 1e-3) / 1e12 / peak, 3),
                                   "note": f"mean of {reps}; inputs ({wg.H}+2x{wg.H_kv} heads) fit in L2"}
         del qg, kg, vg, dog, og, lg, wsg, grads
+        # merge of a 4-way key split of the step's workload (HBM-bound): reads four
+        # [B,H,N,D] bf16 parts and their lse, writes the merged o and lse
+        R = 4
+        parts_o = [torch.randn(w.B, w.H, w.Nq, w.D, device=dev).to(torch.bfloat16) for _ in range(R)]
+        parts_l = [torch.randn(w.B, w.H, w.Nq, device=dev) for _ in range(R)]
+        oc = torch.empty_like(parts_o[0])
+        lc = torch.empty_like(parts_l[0])
+        for _ in range(3):
+            m.mea_attn_combine(parts_o, parts_l, oc, lc)
+        reps = 20
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            m.mea_attn_combine(parts_o, parts_l, oc, lc)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) / reps * 1e3
+        byts = (R + 1) * (parts_o[0].numel() * 2 + parts_l[0].numel() * 4)
+        rows[f"combine_{R}way_{w.name}"] = {"us": round(us, 2), "GB/s": round(byts / (us * 1e-6) / 1e9, 1),
+                                             "frac_of_hbm": round(byts / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 3),
+                                             "bytes": byts, "note": "20 back-to-back launches; 272 MB of parts > L2"}
+        del parts_o, parts_l, oc, lc
         # FP8 forward (e4m3 Q, K; bf16 V, O) on the step's workload
         q8, k8, v8, qd8, kd8 = make_inputs_fp8(w, 0)
         q8, k8, v8 = q8.to(dev), k8.to(dev), v8.to(dev)

@@ -50,7 +50,9 @@ __device__ __forceinline__ void store8(float* p, const float (&x)[8]) {
     *reinterpret_cast<float4*>(p + 4) = make_float4(x[4], x[5], x[6], x[7]);
 }
 
-template <typename T>
+// MAXR: the parts this instantiation handles (4, 8 or 16), so that the per-part
+// registers of a small merge stay few and many threads stay resident.
+template <typename T, int MAXR>
 __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
     const int groups = a.D / 8;
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -58,28 +60,32 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
     const long long row = idx / groups;
     const int g = (int)(idx - row * groups);
 
-    float lv[kCombineMaxParts];
+    float lv[MAXR];
     float M = -INFINITY;
 #pragma unroll
-    for (int r = 0; r < kCombineMaxParts; ++r) {
+    for (int r = 0; r < MAXR; ++r) {
         lv[r] = (r < a.R) ? a.lse_parts[r][row] : -INFINITY;
         M = fmaxf(M, lv[r]);
     }
+    // every part's piece is loaded before any weight is known (one round trip
+    // to memory); a part without keys (lse = -inf, weight 0) is then dropped by
+    // a select, so whatever its o holds (even NaN) never reaches the result
+    float x[MAXR][8];
+#pragma unroll
+    for (int r = 0; r < MAXR; ++r)
+        if (r < a.R) load8(static_cast<const T*>(a.o_parts[r]) + row * a.D + 8 * g, x[r]);
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
     float L = 0.f;
 #pragma unroll
-    for (int r = 0; r < kCombineMaxParts; ++r) {
+    for (int r = 0; r < MAXR; ++r) {
         if (r < a.R) {
-            const float w = ex2_approx((lv[r] - M) * kLog2e);   // 0 for a part without keys (lse = -inf)
-            if (w != 0.f) {
-                float x[8];
-                load8(static_cast<const T*>(a.o_parts[r]) + row * a.D + 8 * g, x);
+            const float w = ex2_approx((lv[r] - M) * kLog2e);
+            const bool use = w != 0.f;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, x[i], acc[i]);
-                L += w;
-            }
+            for (int i = 0; i < 8; ++i) acc[i] = use ? fmaf(w, x[r][i], acc[i]) : acc[i];
+            L += w;
         }
     }
     const float inv = 1.f / L;
@@ -96,10 +102,16 @@ cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t stream)
     if (threads == 0) return cudaSuccess;
     const long long blocks = (threads + 255) / 256;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-    if (bf16)
-        combine_kernel<uint16_t><<<(unsigned)blocks, 256, 0, stream>>>(a);
-    else
-        combine_kernel<float><<<(unsigned)blocks, 256, 0, stream>>>(a);
+    auto run = [&](auto kern) { kern<<<(unsigned)blocks, 256, 0, stream>>>(a); };
+    if (bf16) {
+        if (a.R <= 4) run(combine_kernel<uint16_t, 4>);
+        else if (a.R <= 8) run(combine_kernel<uint16_t, 8>);
+        else run(combine_kernel<uint16_t, kCombineMaxParts>);
+    } else {
+        if (a.R <= 4) run(combine_kernel<float, 4>);
+        else if (a.R <= 8) run(combine_kernel<float, 8>);
+        else run(combine_kernel<float, kCombineMaxParts>);
+    }
     return cudaGetLastError();
 }
 
