@@ -40,6 +40,9 @@
  *    accumulation fp32 (tcgen05 tensor cores).
  *  - MEA_DTYPE_F32: forward and backward, D in {32, 64, 96, 128}; fp32
  *    throughout (SIMT kernels, no tensor cores).
+ *  - e4m3 queries and keys with bf16 values and output: mea_attn_fwd_fp8, D = 128.
+ *  - Key/value heads shared by groups of query heads: the _gqa entry points.
+ *  - Results over disjoint key ranges (a key split) merged: mea_attn_combine.
  *  - Any Nq >= 0 and Nk >= 1; partial tiles are masked.  No mask, no dropout.
  *  - B*H <= 2^31-1 and B*H*max(Nq,Nk)*D < 2^40 elements.
  */
