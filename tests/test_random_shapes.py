@@ -1,0 +1,73 @@
+"""Seeded random shapes through every entry point, against the fp64 oracle (GPU).
+
+Sixty cases drawn from a fixed seed: B in 1..2, H_kv in 1..3 key/value heads
+shared by 1, 2 or 4 query heads, Nq in {1, small, large}, Nk in {1, small,
+large}, D in {64, 128}.  Each runs the bf16 forward and backward; every third
+D = 128 case also runs the FP8 forward and every fourth D = 64 case the fp32
+forward and backward.  Tolerances are those of the dedicated tests, taken
+relative to the largest reference value where outputs are not of order one.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synthetic_inputs import custom, dequant_f64, make_inputs, make_inputs_fp8, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def cases(n=60, seed=2024):
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        D = int(rng.choice([64, 128]))
+        B = int(rng.integers(1, 3))
+        Hkv = int(rng.integers(1, 4))
+        G = int(rng.choice([1, 1, 2, 4]))
+        Nq = int(rng.choice([1, int(rng.integers(1, 40)), int(rng.integers(100, 1200))]))
+        Nk = int(rng.choice([1, int(rng.integers(2, 300)), int(rng.integers(300, 2500))]))
+        out.append((i, B, Hkv * G, Hkv, Nq, Nk, D))
+    return out
+
+
+def rel_max(g, r):
+    g = g.detach().double().cpu().numpy()
+    assert np.isfinite(g).all(), "non-finite values"
+    return float(np.abs(g - r).max() / (1.0 + np.abs(r).max()))
+
+
+@pytest.mark.parametrize("case", cases(), ids=lambda c: "-".join(map(str, c)))
+def test_random_shape(case):
+    import exact_memory_efficient_b200 as m
+    i, B, H, Hkv, Nq, Nk, D = case
+    w = custom(B, H, Nq, Nk, D, "bf16", Hkv=Hkv)
+    q, k, v, do = make_inputs(w, 1000 + i)
+    qd, kd, vd, dod = (x.cuda() for x in (q, k, v, do))
+    o, lse = m.attention_forward(qd, kd, vd, w.scale)
+    dq, dk, dv = m.attention_backward(qd, kd, vd, o, lse, dod, w.scale)
+    assert m.mea_last_device_error() == m.MEA_OK
+    rq, rk, rv, ro, rl = oracle.attention_backward_gqa(to_f64(q), to_f64(k), to_f64(v), to_f64(do), w.scale)
+    assert rel_max(o, ro) < 2e-2
+    assert rel_max(lse, rl) < 1e-3
+    for g_, r_ in ((dq, rq), (dk, rk), (dv, rv)):
+        assert rel_max(g_, r_) < 3e-2
+    if D == 128 and i % 3 == 0:
+        q8, k8, v8, qs, ks = make_inputs_fp8(w, 1000 + i)
+        o8 = torch.empty((B, H, Nq, D), dtype=torch.bfloat16, device="cuda")
+        l8 = torch.empty((B, H, Nq), dtype=torch.float32, device="cuda")
+        m.mea_attn_fwd_fp8(q8.cuda(), k8.cuda(), v8.cuda(), o8, l8, w.scale, qs, ks)
+        assert m.mea_last_device_error() == m.MEA_OK
+        r8, _ = oracle.attention_forward_gqa(dequant_f64(q8, qs), dequant_f64(k8, ks), to_f64(v8), w.scale)
+        assert rel_max(o8, r8) < 2e-2
+    if D == 64 and i % 4 == 0:
+        w32 = custom(B, H, Nq, Nk, D, "f32", Hkv=Hkv)
+        q3, k3, v3, do3 = make_inputs(w32, 1000 + i)
+        qd3, kd3, vd3, dod3 = (x.cuda() for x in (q3, k3, v3, do3))
+        o3, l3 = m.attention_forward(qd3, kd3, vd3, w32.scale)
+        dq3, dk3, dv3 = m.attention_backward(qd3, kd3, vd3, o3, l3, dod3, w32.scale)
+        assert m.mea_last_device_error() == m.MEA_OK
+        r3 = oracle.attention_backward_gqa(to_f64(q3), to_f64(k3), to_f64(v3), to_f64(do3), w32.scale)
+        for g_, r_ in ((o3, r3[3]), (dq3, r3[0]), (dk3, r3[1]), (dv3, r3[2])):
+            assert rel_max(g_, r_) < 1e-4
