@@ -72,7 +72,8 @@ WORKLOADS = {
 }
 WORKLOADS["decode_16384_bf16"] = Workload("decode_16384_bf16", 1, 8, 1, 16384, 128, "bf16", False,
                                           note="decode-shaped bf16 forward: one query row over 16384 keys, 8 heads")
-# Shared key/value heads, with the grouping the survey page gives as its example
+# Shared key/value heads, with the grouping that "当注意力成为瓶颈" (section 推理优化：减少KV Cache)
+# gives as its example
 # (32 query heads in 8 groups of 4).
 WORKLOADS["gqa_32x8_4096_bf16"] = Workload("gqa_32x8_4096_bf16", 1, 32, 4096, 4096, 128, "bf16", True, Hkv=8,
                                            note="grouped-query attention: 32 query heads, 8 key/value heads")
