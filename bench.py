@@ -429,9 +429,11 @@ def run_ours(args):
         # HBM-bound decode-shaped forwards.  Their K/V (67 MB) fit in L2, so each
         # is timed over three copies of its inputs (201 MB > L2) used in turn:
         # every launch reads K/V that the previous two launches evicted.  One
-        # event pair brackets 30 back-to-back launches queued behind a sleep
+        # event pair brackets 30 back-to-back calls queued behind a sleep
         # kernel, so the time is the kernels' (plus the gaps between
-        # consecutive launches), not the host's launch path.
+        # consecutive launches), not the host's launch path.  The row's figure
+        # is the split-KV entry (mea_attn_decode, caller workspace); the
+        # workspace-free forward entry on the same inputs is reported beside it.
         for wname in ("single_query_f32", "decode_16384_bf16", "decode_gqa_32x8_16384_bf16"):
             wd = make_workload(wname)
             sets = []
@@ -439,24 +441,31 @@ def run_ours(args):
                 qd, kd, vd, _ = (x.to(dev) if x is not None else None for x in make_inputs(wd, copy))
                 od, ld = m.attention_forward(qd, kd, vd, wd.scale)
                 sets.append((qd, kd, vd, od, ld))
-            for qd, kd, vd, od, ld in sets:
-                m.mea_attn_fwd_gqa(qd, kd, vd, od, ld, wd.scale)
-            reps = 30
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            torch.cuda.synchronize()
-            torch.cuda._sleep(40_000_000)
-            e0.record(stream)
-            for r in range(reps):
-                qd, kd, vd, od, ld = sets[r % 3]
-                m.mea_attn_fwd_gqa(qd, kd, vd, od, ld, wd.scale)
-            e1.record(stream)
-            torch.cuda.synchronize()
-            us = e0.elapsed_time(e1) / reps * 1e3
+            ws_n = m.mea_attn_decode_workspace_size(wd.B, wd.H, wd.H_kv, wd.Nq, wd.Nk, wd.D, wd.torch_dtype)
+            wsd = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=dev)
+
+            def time_calls(call, reps=30):
+                for st in sets:
+                    call(*st)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize()
+                torch.cuda._sleep(40_000_000)
+                e0.record(stream)
+                for r in range(reps):
+                    call(*sets[r % 3])
+                e1.record(stream)
+                torch.cuda.synchronize()
+                return e0.elapsed_time(e1) / reps * 1e3
+
+            us = time_calls(lambda q_, k_, v_, o_, l_: m.mea_attn_decode(q_, k_, v_, o_, l_, wd.scale, wsd))
+            us_fwd = time_calls(lambda q_, k_, v_, o_, l_: m.mea_attn_fwd_gqa(q_, k_, v_, o_, l_, wd.scale))
             byts = sum(x.numel() * x.element_size() for x in sets[0])
             rows[f"{wname}_fwd"] = {"us": round(us, 2), "GB/s": round(byts / (us * 1e-6) / 1e9, 1),
                                     "frac_of_hbm": round(byts / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 3),
-                                    "bytes": byts, "H_kv": wd.H_kv,
-                                    "note": "30 back-to-back launches over 3 input copies (201 MB > L2)"}
+                                    "bytes": byts, "H_kv": wd.H_kv, "entry": "mea_attn_decode",
+                                    "workspace_bytes": ws_n,
+                                    "mea_attn_fwd_gqa_us": round(us_fwd, 2),
+                                    "note": "30 back-to-back calls over 3 input copies (201 MB > L2)"}
             del sets
         # grouped-query forward + backward (32 query heads over 8 key/value heads)
         wg = make_workload("gqa_32x8_4096_bf16")

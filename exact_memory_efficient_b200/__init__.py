@@ -29,7 +29,8 @@ __all__ = [
     "MEA_BWD_ALL", "MEA_BWD_PREPROCESS", "MEA_BWD_MAIN", "MEA_BWD_FINALIZE",
     "mea_attn_fwd", "mea_attn_bwd", "mea_attn_bwd_phase", "mea_attn_bwd_workspace_size", "mea_attn_bwd_noalloc",
     "mea_attn_fwd_gqa", "mea_attn_bwd_gqa", "mea_attn_bwd_gqa_workspace_size", "mea_attn_fwd_fp8",
-    "mea_attn_combine", "mea_last_device_error",
+    "mea_attn_combine", "mea_attn_decode", "mea_attn_decode_workspace_size", "attention_decode",
+    "mea_last_device_error",
     "mea_selftest_bounded_wait", "mea_status_string", "mea_last_error_message", "mea_version", "attention_forward", "attention_backward",
 ]
 
@@ -97,6 +98,10 @@ def load_library() -> ctypes.CDLL:
     lib.mea_attn_fwd_fp8.restype = i
     lib.mea_attn_combine.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i, vp, vp, i, i, i, i, i, vp]
     lib.mea_attn_combine.restype = i
+    lib.mea_attn_decode_workspace_size.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(sz)]
+    lib.mea_attn_decode_workspace_size.restype = i
+    lib.mea_attn_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, sz, vp]
+    lib.mea_attn_decode.restype = i
     lib.mea_selftest_bounded_wait.argtypes = [vp, vp]
     lib.mea_selftest_bounded_wait.restype = i
     lib.mea_last_device_error.argtypes = [vp]
@@ -297,6 +302,48 @@ def mea_attn_combine(o_parts, lse_parts, o, lse, stream=None) -> None:
     st = load_library().mea_attn_combine(optr, lptr, R, _ptr(o), _ptr(lse), B, H, Nq, D, _dtype_code(o),
                                           _stream_handle(stream))
     _check(st, "mea_attn_combine")
+
+
+def mea_attn_decode_workspace_size(B: int, H: int, H_kv: int, Nq: int, Nk: int, D: int,
+                                   dtype=torch.bfloat16) -> int:
+    """C ``mea_attn_decode_workspace_size`` (for the current CUDA device)."""
+    out = ctypes.c_size_t(0)
+    code = MEA_DTYPE_BF16 if dtype == torch.bfloat16 else MEA_DTYPE_F32
+    st = load_library().mea_attn_decode_workspace_size(B, H, H_kv, Nq, Nk, D, code, ctypes.byref(out))
+    _check(st, "mea_attn_decode_workspace_size")
+    return int(out.value)
+
+
+def mea_attn_decode(q, k, v, o, lse, scale: float, workspace, stream=None) -> None:
+    """C ``mea_attn_decode``: the split-KV forward for few query rows per key/value head.  Shapes as
+    for ``mea_attn_fwd_gqa``; ``workspace`` a CUDA tensor of at least
+    ``mea_attn_decode_workspace_size`` bytes (None when that size is 0)."""
+    B, H, Hkv, Nq, Nk, D = _gqa_shapes(q, k, "mea_attn_decode")
+    if tuple(v.shape) != tuple(k.shape) or tuple(o.shape) != tuple(q.shape):
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_decode: shape mismatch")
+    if tuple(lse.shape) != (B, H, Nq) or lse.dtype != torch.float32:
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_decode: lse must be fp32 [B, H, Nq]")
+    if not (q.dtype == k.dtype == v.dtype == o.dtype):
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_decode: dtype mismatch")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load_library().mea_attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Nq, Nk, D,
+                                         float(scale), _dtype_code(q), _ptr(workspace), ws_bytes,
+                                         _stream_handle(stream))
+    _check(st, "mea_attn_decode")
+
+
+def attention_decode(q, k, v, scale: float | None = None, stream=None):
+    """Allocate (o, lse) and the workspace with torch and run ``mea_attn_decode``."""
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    B, H, Nq, D = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    n = mea_attn_decode_workspace_size(B, H, Hkv, Nq, Nk, D, q.dtype)
+    ws = torch.empty(n, dtype=torch.uint8, device=q.device) if n else None
+    mea_attn_decode(q, k, v, o, lse, scale, ws, stream)
+    return o, lse
 
 
 def mea_selftest_bounded_wait(gave_up, stream=None) -> None:

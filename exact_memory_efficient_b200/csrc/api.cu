@@ -211,6 +211,51 @@ mea_status_t tc_forward(const void* q, const void* k, const void* v, void* o, fl
     return cuda_status(mea::launch_fwd_bf16(a, s), "fwd_bf16 launch");
 }
 
+// Split-KV decode plan for BHkv key/value heads of R query rows each: the key
+// range of a head is cut into nsplit chunks of whole 64-key tiles so that the
+// launch has at most one CTA per slot of the device (SMs x resident CTAs of
+// the partial kernel) and every chunk holds at least one key.
+struct DecodePlan {
+    int nsplit = 1;
+    int chunk_len = 0;
+    size_t ws_bytes = 0;   // chunk summaries; 0 when nsplit == 1
+};
+DecodePlan decode_plan(const DeviceInfo* dev, long long BHkv, int R, int Nk, int D, bool bf16) {
+    DecodePlan p;
+    const long long tiles = ((long long)Nk + mea::kDecodeTileKeys - 1) / mea::kDecodeTileKeys;
+    const long long slots = (long long)dev->sm_count * mea::decode_blocks_per_sm(bf16, D, R);
+    long long n = 1;
+    if (BHkv > 0 && BHkv < slots) n = slots / BHkv;
+    if (n > tiles) n = tiles;
+    if (n < 1) n = 1;
+    const long long chunk_tiles = (tiles + n - 1) / n;
+    p.nsplit = (int)((tiles + chunk_tiles - 1) / chunk_tiles);
+    p.chunk_len = (int)(chunk_tiles * mea::kDecodeTileKeys);
+    if (p.nsplit > 1) p.ws_bytes = (size_t)BHkv * p.nsplit * R * (D + 2) * sizeof(float);
+    return p;
+}
+
+mea_status_t launch_decode_plan(const void* q, const void* k, const void* v, void* o, float* lse, long long BHkv,
+                                int R, int Nk, int D, float scale, bool bf16, const DecodePlan& p, void* ws,
+                                cudaStream_t s) {
+    mea::DecodeArgs a;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.o = o;
+    a.lse = lse;
+    a.BHkv = BHkv;
+    a.R = R;
+    a.Nk = Nk;
+    a.D = D;
+    a.scale = scale;
+    a.nsplit = p.nsplit;
+    a.chunk_len = p.chunk_len;
+    a.part_acc = static_cast<float*>(ws);
+    a.part_ml = p.nsplit > 1 ? a.part_acc + (size_t)BHkv * p.nsplit * R * D : nullptr;
+    return cuda_status(mea::launch_decode(a, bf16, s), "decode launch");
+}
+
 mea_status_t common_checks(int B, int H, int Nq, int Nk, int D, float scale, mea_dtype_t dtype) {
     if (dtype != MEA_DTYPE_F32 && dtype != MEA_DTYPE_BF16) return MEA_ERR_INVALID_ARG;
     if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || D <= 0) return MEA_ERR_INVALID_ARG;
@@ -258,6 +303,14 @@ mea_status_t mea_attn_fwd(const void* q, const void* k, const void* v, void* o, 
     if ((st = device_info(&dev)) != MEA_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int BH = B * H;
+
+    // Few rows per head: when one chunk per head already fills the device, the
+    // split-KV decode kernel runs alone (no workspace needed).
+    const bool bf16 = dtype == MEA_DTYPE_BF16;
+    if (mea::decode_supported(bf16, D, Nq)) {
+        const DecodePlan p = decode_plan(dev, BH, Nq, Nk, D, bf16);
+        if (p.nsplit == 1) return launch_decode_plan(q, k, v, o, lse, BH, Nq, Nk, D, scale, bf16, p, nullptr, s);
+    }
 
     if (dtype == MEA_DTYPE_F32) {
         mea::F32FwdArgs a;
@@ -433,6 +486,50 @@ mea_status_t mea_attn_fwd_gqa(const void* q, const void* k, const void* v, void*
     mea_status_t st = gqa_rows(H, H_kv, Nq, &rows);
     if (st != MEA_OK) return st;
     return mea_attn_fwd(q, k, v, o, lse, B, H_kv, rows, Nk, D, scale, dtype, stream);
+}
+
+mea_status_t mea_attn_decode_workspace_size(int B, int H, int H_kv, int Nq, int Nk, int D, mea_dtype_t dtype,
+                                          size_t* bytes) {
+    if (bytes == nullptr) return MEA_ERR_INVALID_ARG;
+    int rows = 0;
+    mea_status_t st = gqa_rows(H, H_kv, Nq, &rows);
+    if (st != MEA_OK) return st;
+    if ((st = common_checks(B, H_kv, rows, Nk, D, 1.0f, dtype)) != MEA_OK) return st;
+    *bytes = 0;
+    const bool bf16 = dtype == MEA_DTYPE_BF16;
+    if ((long long)B * H_kv * rows == 0 || Nk == 0 || !mea::decode_supported(bf16, D, rows)) return MEA_OK;
+    DeviceInfo* dev = nullptr;
+    if ((st = device_info(&dev)) != MEA_OK) return st;
+    *bytes = decode_plan(dev, (long long)B * H_kv, rows, Nk, D, bf16).ws_bytes;
+    return MEA_OK;
+}
+
+mea_status_t mea_attn_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                             int H_kv, int Nq, int Nk, int D, float scale, mea_dtype_t dtype, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+    int rows = 0;
+    mea_status_t st = gqa_rows(H, H_kv, Nq, &rows);
+    if (st != MEA_OK) return st;
+    const bool bf16 = dtype == MEA_DTYPE_BF16;
+    if (dtype != MEA_DTYPE_F32 && dtype != MEA_DTYPE_BF16) return MEA_ERR_INVALID_ARG;
+    if (!mea::decode_supported(bf16, D, rows))   // many rows per head: the tensor-core / fp32 forward
+        return mea_attn_fwd(q, k, v, o, lse, B, H_kv, rows, Nk, D, scale, dtype, stream);
+    if ((st = common_checks(B, H_kv, rows, Nk, D, scale, dtype)) != MEA_OK) return st;
+    const long long BHkv = (long long)B * H_kv;
+    if (BHkv * rows == 0) return MEA_OK;
+    if (Nk == 0) return MEA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !o || !lse) return MEA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse)) return MEA_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    if ((st = device_info(&dev)) != MEA_OK) return st;
+    const DecodePlan p = decode_plan(dev, BHkv, rows, Nk, D, bf16);
+    if (p.nsplit > 1) {
+        if (workspace == nullptr || workspace_bytes < p.ws_bytes)
+            return fail(MEA_ERR_WORKSPACE, "mea_attn_decode", "workspace missing or below mea_attn_decode_workspace_size");
+        if (!aligned16(workspace)) return MEA_ERR_MISALIGNED;
+    }
+    return launch_decode_plan(q, k, v, o, lse, BHkv, rows, Nk, D, scale, bf16, p, workspace,
+                              static_cast<cudaStream_t>(stream));
 }
 
 mea_status_t mea_attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,

@@ -39,7 +39,7 @@ struct CombineArgs {
 };
 cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t stream);
 
-// fp32 SIMT backward (bwd_f32.cu).// fp32 SIMT backward (bwd_f32.cu).  Row term D_i in `delta` (workspace).
+// fp32 SIMT backward (bwd_f32.cu).  Row term D_i in `delta` (workspace).
 struct F32BwdArgs {
     const float* q;
     const float* k;
@@ -57,6 +57,31 @@ struct F32BwdArgs {
     int k_rows_per_cta;  // dK/dV kernel: key rows per CTA of 8 warps (1, 2, 4 or 8)
 };
 cudaError_t launch_bwd_f32(const F32BwdArgs& a, cudaStream_t stream, unsigned phases);
+
+// Split-KV forward for few query rows per key/value head (decode.cu).  q, o
+// are [BHkv, R, D] (the R = G*Nq rows sharing one key/value head), k, v are
+// [BHkv, Nk, D], bf16 or fp32.  With nsplit > 1 the chunk summaries go to
+// part_acc [BHkv, nsplit, R, D] and part_ml [BHkv, nsplit, R, 2] (fp32) and a
+// second kernel merges them; with nsplit == 1 the first kernel writes o, lse.
+constexpr int kDecodeMaxRows = 8;
+constexpr int kDecodeTileKeys = 64;
+struct DecodeArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    void* o;
+    float* lse;
+    float* part_acc;
+    float* part_ml;
+    long long BHkv;
+    int R, Nk, D;
+    float scale;
+    int nsplit;     // key chunks per key/value head (grid y)
+    int chunk_len;  // keys per chunk (multiple of kDecodeTileKeys)
+};
+bool decode_supported(bool bf16, int D, int R);
+int decode_blocks_per_sm(bool bf16, int D, int R);   // CTAs of the partial kernel per SM
+cudaError_t launch_decode(const DecodeArgs& a, bool bf16, cudaStream_t stream);
 
 // bf16 tcgen05 forward (fwd_bf16.cu).  Tensor maps are 3-D {D, N, B*H} bf16,
 // 128-byte swizzle, box {64, 128, 1}.

@@ -23,7 +23,7 @@
  *    lse: [B, H, Nq] fp32 (natural log of the scaled scores' exp-sum).
  *  - Every pointer is caller-owned DEVICE memory.  The library never
  *    allocates, frees or synchronises inside fwd/bwd; scratch memory for the
- *    backward pass is the caller's `workspace`.
+ *    backward pass and the split-KV decode is the caller's `workspace`.
  *  - Tensor pointers (q, k, v, o, dO, dq, dk, dv, workspace) must be 16-byte
  *    aligned; lse must be 4-byte aligned.
  *  - `stream` is a cudaStream_t (CUstream) passed as void*; NULL means the
@@ -43,6 +43,8 @@
  *  - e4m3 queries and keys with bf16 values and output: mea_attn_fwd_fp8, D = 128.
  *  - Key/value heads shared by groups of query heads: the _gqa entry points.
  *  - Results over disjoint key ranges (a key split) merged: mea_attn_combine.
+ *  - Decode-shaped calls (at most 8 query rows per key/value head) over all
+ *    SMs with a caller-given workspace: mea_attn_decode.
  *  - Any Nq >= 0 and Nk >= 1; partial tiles are masked.  No mask, no dropout.
  *  - B*H <= 2^31-1 and B*H*max(Nq,Nk)*D < 2^40 elements.
  */
@@ -249,6 +251,46 @@ mea_status_t mea_attn_fwd_fp8(const void* q, const void* k, const void* v,
 mea_status_t mea_attn_combine(const void* const* o_parts, const float* const* lse_parts, int R,
                               void* o, float* lse, int B, int H, int Nq, int D,
                               mea_dtype_t dtype, void* stream);
+
+/*
+ * Split-KV forward for decode-shaped calls: few query rows per key/value head
+ * against a long key range (token-by-token generation).
+ *
+ * Source: "Self-attention Does Not Need O(n^2) Memory" (Chinese summary,
+ * section 方法详解: for a single query the scores and weighted values are
+ * accumulated key by key with two running quantities, the weighted sum and the
+ * total weight, plus the running maximum), its chunk summaries merged with the
+ * two-block formulas of "当注意力成为瓶颈从on困境到线性复杂度的技术突围"
+ * (section IO感知); the workload is the one the "overhead" page (section
+ * 对模型开发与部署的影响) names for autoregressive generation, where every new
+ * token attends to all previous ones.  The operation is exactly that of
+ * mea_attn_fwd_gqa.
+ *
+ * With R = (H / H_kv) * Nq <= 8 rows per key/value head (and a head dim of the
+ * dtype's supported set) the call reads K and V once with every SM of the
+ * device: the keys of each head are cut into chunks, every CTA summarises one
+ * chunk (running max, exp-sum, unnormalised fp32 accumulator) into
+ * `workspace`, and a second kernel merges the summaries into o and lse.  With
+ * more rows per head the call is mea_attn_fwd_gqa and `workspace` is unused.
+ *
+ * Arguments, layouts, alignment and dtypes are those of mea_attn_fwd_gqa.
+ * workspace: caller-owned device memory of at least the size that
+ * mea_attn_decode_workspace_size returns for the same shape on the device
+ * current at the call (it depends on the device's SM count); 16-byte aligned;
+ * its contents are scratch (no initialisation needed, nothing kept).  Size 0
+ * (workspace may be NULL) when one chunk per head already fills the device or
+ * the call has more than 8 rows per head.
+ * Errors: those of mea_attn_fwd_gqa, plus MEA_ERR_WORKSPACE (missing or too
+ * small) and MEA_ERR_MISALIGNED for the workspace.
+ */
+mea_status_t mea_attn_decode_workspace_size(int B, int H, int H_kv, int Nq, int Nk, int D,
+                                            mea_dtype_t dtype, size_t* bytes);
+
+mea_status_t mea_attn_decode(const void* q, const void* k, const void* v,
+                             void* o, float* lse,
+                             int B, int H, int H_kv, int Nq, int Nk, int D, float scale,
+                             mea_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                             void* stream);
 
 /*
  * Backward pass that allocates nothing and takes no workspace.  The paper has

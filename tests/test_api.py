@@ -202,3 +202,32 @@ def test_combine_argument_validation(lib):
     assert comb(lptr=A + 2) == 3
     assert comb(o=A + 4) == 3
     assert comb(Nq=0) == 0                 # nothing to merge
+
+
+def test_decode_argument_validation(lib):
+    def dec(q=A, k=A, v=A, o=A, lse=A, B=1, H=8, Hkv=8, Nq=1, Nk=1024, D=128, scale=0.125, dtype=BF16,
+            ws=A, ws_bytes=1 << 20):
+        return lib.mea_attn_decode(q, k, v, o, lse, B, H, Hkv, Nq, Nk, D, ctypes.c_float(scale), dtype, ws,
+                                   ws_bytes, None)
+
+    assert dec(q=None) == 1
+    assert dec(lse=None) == 1
+    assert dec(Hkv=3) == 1                 # H not a multiple of H_kv
+    assert dec(Hkv=0) == 1
+    assert dec(Nk=0) == 1
+    assert dec(scale=float("nan")) == 1
+    assert dec(dtype=7) == 1
+    assert dec(D=96) == 2                  # bf16 head dims are 64 and 128
+    assert dec(D=96, dtype=F32, q=A + 8) == 3
+    assert dec(k=A + 8) == 3
+    assert dec(lse=A + 2) == 3
+    assert dec(Nq=0) == 0                  # no rows: no-op
+    assert dec(B=0) == 0
+    assert dec(Nq=16, q=None) == 1         # 16 rows per head: the mea_attn_fwd_gqa path, same checks
+    size = ctypes.c_size_t(99)
+    # more than 8 rows per head: no split, no workspace (answered without a device)
+    assert lib.mea_attn_decode_workspace_size(1, 8, 8, 16, 1024, 128, BF16, ctypes.byref(size)) == 0
+    assert size.value == 0
+    assert lib.mea_attn_decode_workspace_size(1, 8, 3, 1, 1024, 128, BF16, ctypes.byref(size)) == 1
+    assert lib.mea_attn_decode_workspace_size(1, 8, 8, 1, 1024, 128, BF16, None) == 1
+    assert lib.mea_attn_decode_workspace_size(1, 8, 8, 1, 1024, 96, BF16, ctypes.byref(size)) == 2
