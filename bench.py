@@ -581,15 +581,19 @@ def run_ours(args):
 
 
 def run_profile(name: str) -> int:
-    """Three forward (+ backward) calls of one workload through the public API, untimed."""
+    """Three forward (+ backward) calls of one workload through the public API, untimed.
+    Forward-only workloads go through mea_attn_decode, the entry the decode rows time
+    (it is the plain forward when a head has more than 8 query rows)."""
     import exact_memory_efficient_b200 as m
     w = make_workload(name)
     torch.cuda.set_device(0)
     q, k, v, do = (x.cuda() if x is not None else None for x in make_inputs(w, 0))
     for _ in range(3):
+        if do is None:
+            m.attention_decode(q, k, v, w.scale)
+            continue
         o, lse = m.attention_forward(q, k, v, w.scale)
-        if do is not None:
-            m.attention_backward(q, k, v, o, lse, do, w.scale)
+        m.attention_backward(q, k, v, o, lse, do, w.scale)
     st = m.mea_last_device_error()
     if st != m.MEA_OK:
         raise RuntimeError(m.mea_status_string(st))
@@ -611,7 +615,7 @@ def main():
                     help="skip the end-to-end, fp32-row and CPU-baseline measurements (profiling captures)")
     ap.add_argument("--profile", metavar="WORKLOAD", default=None,
                     help="no timing: run this workload's forward (and backward, if it has one) three times and "
-                         "exit; the command profiling captures wrap")
+                         "exit; the command profiling captures wrap (forward-only workloads: mea_attn_decode)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

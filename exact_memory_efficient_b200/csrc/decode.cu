@@ -33,8 +33,11 @@
 //               lse, otherwise the chunk summary (m, l, acc) goes to the
 //               caller's workspace.
 // Phase 2, decode_merge_kernel: merges the nsplit chunk summaries of each row.
-// It is launched with programmatic stream serialisation: its CTAs may start
-// while phase 1 drains and wait (griddepcontrol.wait) for phase 1's results.
+// Both kernels are launched with programmatic stream serialisation: a grid may
+// be scheduled while the kernel before it in the stream drains, and waits
+// (griddepcontrol.wait) for that kernel's results before it touches global
+// memory, so results are as with plain stream order while the launch and
+// set-up of one kernel overlap the tail of the previous one.
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -114,6 +117,36 @@ __device__ __forceinline__ void store_out(uint16_t* p, float x) {
 }
 __device__ __forceinline__ void store_out(float* p, float x) { *p = x; }
 
+// (d0, d1) += (a0, a1) * (b0, b1) as one packed fp32 FMA (each lane rounded as fmaf)
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 pa, pb, pd;\n\t"
+        "mov.b64 pa, {%2, %3};\n\t"
+        "mov.b64 pb, {%4, %5};\n\t"
+        "mov.b64 pd, {%0, %1};\n\t"
+        "fma.rn.f32x2 pd, pa, pb, pd;\n\t"
+        "mov.b64 {%0, %1}, pd;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// Dot product of DPL-element slices: pairs through the packed FMA.
+template <int DPL>
+__device__ __forceinline__ float dot_slice(const float (&a)[DPL], const float (&b)[DPL]) {
+    float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+    for (int i = 0; i + 1 < DPL; i += 2) fma2(d0, d1, a[i], a[i + 1], b[i], b[i + 1]);
+    if constexpr (DPL % 2 == 1) d0 = fmaf(a[DPL - 1], b[DPL - 1], d0);
+    return d0 + d1;
+}
+
+// acc += p * v over a DPL-element slice, pairs through the packed FMA.
+template <int DPL>
+__device__ __forceinline__ void axpy_slice(float (&acc)[DPL], float p, const float (&v)[DPL]) {
+#pragma unroll
+    for (int i = 0; i + 1 < DPL; i += 2) fma2(acc[i], acc[i + 1], p, p, v[i], v[i + 1]);
+    if constexpr (DPL % 2 == 1) acc[DPL - 1] = fmaf(p, v[DPL - 1], acc[DPL - 1]);
+}
+
 // Butterfly reduce-scatter of N values (N = 8, 16 or 32) over the 32 lanes:
 // on return the lane holds the warp-wide sum of value v = lane >> (5 - log2 N).
 // Each halving step exchanges half of the remaining values with the partner
@@ -170,6 +203,10 @@ decode_partial_kernel(const DecodeArgs a) {
         fence_mbar_init();
     }
     __syncthreads();
+    // This grid may have been launched before the previous kernel of the stream
+    // finished (programmatic stream serialisation): nothing global is touched
+    // before that kernel's results are complete and visible.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // the merge kernel may be scheduled from now on; it waits for this grid's results
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
@@ -242,12 +279,7 @@ decode_partial_kernel(const DecodeArgs a) {
 #pragma unroll
                 for (int j = 0; j < kKeysPerWarp; ++j)
 #pragma unroll
-                    for (int rr = 0; rr < RR; ++rr) {
-                        float d = 0.f;
-#pragma unroll
-                        for (int i = 0; i < DPL; ++i) d = fmaf(qr[p * RR + rr][i], kf[j][i], d);
-                        part[j * RR + rr] = d;
-                    }
+                    for (int rr = 0; rr < RR; ++rr) part[j * RR + rr] = dot_slice<DPL>(qr[p * RR + rr], kf[j]);
                 float sv = reduce_scatter<C::kN>(part, lane);
                 sv = (j_mine < valid) ? sv : -INFINITY;
                 float& m = m_mine[p];
@@ -278,8 +310,7 @@ decode_partial_kernel(const DecodeArgs a) {
 #pragma unroll
                         for (int rr = 0; rr < RR; ++rr) {
                             const float pj = __shfl_sync(0xffffffffu, pw, (j * RR + rr) << kSh);
-#pragma unroll
-                            for (int i = 0; i < DPL; ++i) acc[p * RR + rr][i] = fmaf(pj, vf[i], acc[p * RR + rr][i]);
+                            axpy_slice<DPL>(acc[p * RR + rr], pj, vf);
                         }
                     }
                 }
@@ -366,6 +397,8 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const Decod
     __shared__ float s_m[kMergeThreads];
     __shared__ float s_l[kMergeThreads];
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // a following launch with programmatic serialisation may start its set-up
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const long long row = blockIdx.x;
     const long long bh = row / a.R;
     const int r = (int)(row - bh * a.R);
@@ -453,7 +486,18 @@ cudaError_t launch_partial(const DecodeArgs& a, cudaStream_t stream) {
     auto kern = decode_partial_kernel<T, DPL, RMAX>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    kern<<<dim3((unsigned)a.BHkv, (unsigned)a.nsplit), kThreads, C::kSmemBytes, stream>>>(a);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)a.BHkv, (unsigned)a.nsplit);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
