@@ -15,8 +15,13 @@
 //                  S^T  = K Q_i^T          (smem x smem -> TMEM)
 //                  dP^T = V dO_i^T         (smem x smem -> TMEM)
 //                  dV  += P^T dO_i         (P^T from TMEM, bf16)
-//                  dK  += dS^T Q_i         (dS^T from TMEM, bf16)
 //                  dQ_i^T = K^T dS^T       (both from smem, bf16) -> fp32 TMA reduce-add
+//                  dK  += dS^T Q_i         (both from smem, bf16)
+//                dS^T is written once, to swizzled shared memory, where it is
+//                the MN-major B operand of dQ^T and the K-major A operand of
+//                dK.  dQ^T is issued before dK, so the dQ warps copy it out of
+//                TMEM (and dP^T of the next tile can take its columns) while
+//                dK runs.
 //                dQ is formed transposed so that TMEM lanes are head dims: each
 //                warp of the dQ warpgroup stages [64 queries x 32 head dims] of
 //                it in shared memory and one TMA reduce-add sends it to the dQ
@@ -31,7 +36,7 @@
 //   warp 1       MMA issuer (one thread)
 //   warps 4-11   two compute warpgroups: thread (warp w, lane) owns key row
 //                32*(w%4)+lane (the TMEM lane warp w can reach) and query half
-//                (w-4)/4 of every tile: P^T and dS^T
+//                (w-4)/4 of every tile: P^T (to TMEM) and dS^T (to smem)
 //   warps 12-15  dQ warpgroup: copies dQ_i^T out of TMEM (freeing it at once),
 //                stages it in its own shared-memory buffer and hands it to the
 //                TMA engine as fp32 reduce-adds into the dQ accumulator; also
@@ -252,10 +257,12 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             constexpr unsigned idesc_t = make_idesc_bf16(128, 128, 0, 0);   // S^T, dP^T
             constexpr unsigned idesc_g = make_idesc_bf16(128, D, 0, 1);     // dV, dK (A in TMEM)
             constexpr unsigned idesc_q = make_idesc_bf16(128, 128, 1, 1);   // dQ^T (A = K^T, B = dS^T, MN-major)
+            constexpr unsigned idesc_k = make_idesc_bf16(128, D, 0, 1);     // dK (A = dS^T K-major, B = Q MN-major)
             const uint32_t k_lo = desc_lo_kmajor(smem_u32(sK));             // K as A of S^T
             const uint32_t kt_lo = desc_lo_mnmajor(smem_u32(sK));           // K^T as A of dQ^T
             const uint32_t v_lo = desc_lo_kmajor(smem_u32(sV));
-            const uint32_t ds_lo = desc_lo_mnmajor(smem_u32(sDS));
+            const uint32_t ds_lo = desc_lo_mnmajor(smem_u32(sDS));          // dS^T as B of dQ^T
+            const uint32_t dsk_lo = desc_lo_kmajor(smem_u32(sDS));          // dS^T as A of dK
             const uint32_t do_k_lo = desc_lo_kmajor(smem_u32(sDO));         // dO as B of dP^T
             const uint32_t do_mn_lo = desc_lo_mnmajor(smem_u32(sDO));       // dO as B of dV
             const uint32_t q_k_lo0 = desc_lo_kmajor(smem_u32(sQ));
@@ -300,12 +307,10 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     mma_ts_lo(tDV, tS + packed_col(kk), do_mn_lo + mnmajor_step(kk), idesc_g, (acc0 | kk) ? 1u : 0u);
                 mma_commit(&bars->do_empty);           // dO_i read by dP^T(i) and dV(i)
                 if (i + 1 < n_q && !(ok = issue_s(i + 1))) break;
-                // dK += dS^T Q_i ; dQ_i^T = K^T dS^T
+                // dQ_i^T = K^T dS^T first, so the dQ warps copy it out while dK
+                // runs; dK += dS^T Q_i then reads dS^T from shared memory too
                 if (!(ok = mbar_wait(&bars->ds_ready, i & 1, abort_flag))) break;
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk)
-                    mma_ts_lo(tDK, tDP + packed_col(kk), q_mn_lo + mnmajor_step(kk), idesc_g, (acc0 | kk) ? 1u : 0u);
                 if (!Cfg::kDqInDp && i > 0) {
                     if (!(ok = mbar_wait(&bars->dq_free, (i - 1) & 1, abort_flag))) break;
                     tc_fence_after();
@@ -314,6 +319,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int kk = 0; kk < kTile / 16; ++kk)
                     mma_ss_lo(tDQ, kt_lo + mnmajor_step(kk), ds_lo + mnmajor_step(kk), idesc_q, kk > 0);
                 mma_commit(&bars->dq_full);
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    mma_ss_lo(tDK, dsk_lo + kmajor_step(kk), q_mn_lo + mnmajor_step(kk), idesc_k, (acc0 | kk) ? 1u : 0u);
                 mma_commit(&bars->q_empty[i & 1]);
             }
             if (ok) mma_commit(&bars->final_done);
@@ -359,7 +367,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         auto do_ds = [&](int t) -> bool {
             const float* dl = s_delta + (t & 1) * kTile + 64 * g;
             if (!mbar_wait(&bars->dp_full, t & 1, abort_flag)) return false;
-            // dp_full(t) was committed after dQ(t-1), so the dS buffer is free again
+            // dp_full(t) was committed after dQ(t-1) and dK(t-1), the readers of the dS buffer
             tc_fence_after();
             // dS^T (keys x queries) in shared memory: MN-major operand, query block g,
             // row = key, 16-byte chunk c of the 128-byte row swizzled by (key mod 8).
@@ -378,8 +386,6 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     const float d1 = __uint_as_float(pr & 0xffff0000u) * (__uint_as_float(dr[2 * c + 1]) - dl[q + 1]);
                     pk[c] = pack_bf16x2(d0, d1);
                 }
-                // packed dS^T overwrites dP^T columns this thread has already read
-                tmem_st16(tmem + lane_off + Cfg::colDP + 64 * g + 16 * h, pk);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const int pc = (4 * h + c) ^ (kr & 7);
@@ -388,7 +394,6 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             }
             fence_proxy_async_smem();
-            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars->ds_ready);
             return true;
