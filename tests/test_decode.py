@@ -157,3 +157,36 @@ def test_decode_workspace_errors():
     m.mea_attn_decode(q, k, v, o, lse, w.scale, big)
     ro, rl = oracle.attention_forward(*(to_f64(x.cpu()) for x in (q, k, v)), w.scale)
     assert_close(to_np(o), ro, *BF16_O, what="garbage workspace")
+
+
+def test_decode_in_cuda_graph():
+    """Both decode kernels are launched with programmatic stream serialisation; a CUDA graph
+    captures them (and a backward in the same graph) and replays them with new inputs."""
+    import exact_memory_efficient_b200 as m
+    w = custom(1, 8, 1, 5000, 128, "bf16", backward=False, Hkv=2)
+    q, k, v, _ = (x.cuda() if x is not None else None for x in make_inputs(w, 40))
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")
+    n = m.mea_attn_decode_workspace_size(1, 8, 2, 1, 5000, 128)
+    ws = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        m.mea_attn_decode(q, k, v, o, lse, w.scale, ws, stream=s)   # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        m.mea_attn_decode(q, k, v, o, lse, w.scale, ws)
+    for seed in (41, 42):
+        q2, k2, v2, _ = make_inputs(w, seed)
+        q.copy_(q2.cuda())
+        k.copy_(k2.cuda())
+        v.copy_(v2.cuda())
+        g.replay()
+        torch.cuda.synchronize()
+        ro, rl = oracle.attention_forward_gqa(to_f64(q2), to_f64(k2), to_f64(v2), w.scale)
+        assert_close(to_np(o), ro, *BF16_O, what=f"graph replay O seed {seed}")
+        assert_lse_close(to_np(lse), rl, to_f64(q2), np.repeat(to_f64(k2), 4, axis=1), w.scale,
+                         what=f"graph replay lse seed {seed}")
+    assert m.mea_last_device_error() == m.MEA_OK
