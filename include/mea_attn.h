@@ -280,6 +280,10 @@ mea_status_t mea_attn_combine(const void* const* o_parts, const float* const* ls
  * its contents are scratch (no initialisation needed, nothing kept).  Size 0
  * (workspace may be NULL) when one chunk per head already fills the device or
  * the call has more than 8 rows per head.
+ * Both kernels of the split path are launched with programmatic stream
+ * serialisation: a kernel may begin its set-up while the previous kernel in
+ * the stream drains, but reads or writes no global memory before that kernel
+ * has completed, so ordering is that of a plain stream (graph capture works).
  * Errors: those of mea_attn_fwd_gqa, plus MEA_ERR_WORKSPACE (missing or too
  * small) and MEA_ERR_MISALIGNED for the workspace.
  */
