@@ -18,10 +18,12 @@
 //   warp 8      producer: cp.async.bulk copies of 64-key K and V tiles
 //               (contiguous rows of the [B*H_kv, Nk, D] tensors) into the ring.
 //   warps 0-7   warp w takes keys [8w, 8w + 8) of every tile and keeps its own
-//               running (m, l, acc) per row.  Lane l owns head dims
-//               [l*DPL, (l+1)*DPL): it forms partial dot products for its 8
-//               keys x up to 4 rows and a butterfly reduce-scatter leaves every
-//               (key, row) score complete in one group of lanes; the score
+//               running (m, l, acc) per row.  A key is shared by the whole
+//               warp (1 or 8 rows per head) or by a half-warp (2 or 4 rows,
+//               two keys at a time); each lane owns a slice of the head dims,
+//               forms partial dot products for its keys x up to 4 rows, and a
+//               butterfly reduce-scatter over the key's lanes leaves every
+//               (key, row) score complete in one set of lanes; the score
 //               is already in the base-2 domain (q is pre-multiplied by
 //               scale * log2 e).  The maximum is refreshed only when a score
 //               exceeds it by more than 2^8 (the rescale is exact whenever it
@@ -57,9 +59,19 @@ constexpr float kRescaleThreshold = 8.0f;        // log2 of the largest weight l
 
 constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
 
+// Lanes per key: 2 and 4 rows per head put 16 lanes (half a warp) on a key,
+// so a warp reduces two keys' products at once over 16 lanes; 1 and 8 rows use
+// the whole warp (one row's products are few; eight rows need the registers).
+template <int RMAX>
+constexpr int kLanesPerKey = (RMAX == 2 || RMAX == 4) ? 16 : 32;
+
 template <typename T, int DPL, int RMAX>
 struct DecCfg {
     static constexpr int D = 32 * DPL;
+    static constexpr int LPK = kLanesPerKey<RMAX>;
+    static constexpr int kGroups = 32 / LPK;              // key groups per warp (1 or 2)
+    static constexpr int kKPG = kKeysPerWarp / kGroups;   // keys per group in a tile
+    static constexpr int DL = D / LPK;                    // head dims per lane
     static constexpr int kRowBytes = D * (int)sizeof(T);
     static constexpr int kTileBytes = kTK * kRowBytes;   // K or V part of a stage
     static constexpr int kStageBytes = 2 * kTileBytes;
@@ -69,8 +81,8 @@ struct DecCfg {
     static constexpr int kStages = kRingBudget / kStageBytes < 2 ? 2 : kRingBudget / kStageBytes;
     static constexpr int RR = RMAX < 4 ? RMAX : 4;        // rows per pass
     static constexpr int kPasses = RMAX / RR;
-    static constexpr int kN = kKeysPerWarp * RR;          // values per reduce-scatter: 8, 16 or 32
-    static constexpr int kSh = 5 - ilog2(kN);             // lane -> value: v = lane >> kSh
+    static constexpr int kN = kKPG * RR;                  // values per reduce-scatter: 8, 16 or 32
+    static constexpr int kSh = ilog2(LPK) - ilog2(kN);    // lane in group -> value: v = li >> kSh
     // merge scratch over the drained ring: acc, m, l of every warp and row
     static constexpr int kScratchBytes = kCompWarps * RMAX * (D + 2) * 4;
     static constexpr int kRingBytes = kStages * kStageBytes;
@@ -93,6 +105,15 @@ __device__ __forceinline__ void load_row(const uint16_t* p, float (&x)[4]) {
     x[2] = __uint_as_float(u.y << 16);
     x[3] = __uint_as_float(u.y & 0xffff0000u);
 }
+__device__ __forceinline__ void load_row(const uint16_t* p, float (&x)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
 __device__ __forceinline__ void load_row(const float* p, float (&x)[1]) { x[0] = *p; }
 __device__ __forceinline__ void load_row(const float* p, float (&x)[2]) {
     const float2 u = *reinterpret_cast<const float2*>(p);
@@ -110,6 +131,24 @@ __device__ __forceinline__ void load_row(const float* p, float (&x)[4]) {
     x[1] = u.y;
     x[2] = u.z;
     x[3] = u.w;
+}
+__device__ __forceinline__ void load_row(const float* p, float (&x)[6]) {
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+        const float2 u = reinterpret_cast<const float2*>(p)[i];
+        x[2 * i] = u.x;
+        x[2 * i + 1] = u.y;
+    }
+}
+__device__ __forceinline__ void load_row(const float* p, float (&x)[8]) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float4 u = reinterpret_cast<const float4*>(p)[i];
+        x[4 * i] = u.x;
+        x[4 * i + 1] = u.y;
+        x[4 * i + 2] = u.z;
+        x[4 * i + 3] = u.w;
+    }
 }
 
 __device__ __forceinline__ void store_out(uint16_t* p, float x) {
@@ -147,16 +186,18 @@ __device__ __forceinline__ void axpy_slice(float (&acc)[DPL], float p, const flo
     if constexpr (DPL % 2 == 1) acc[DPL - 1] = fmaf(p, v[DPL - 1], acc[DPL - 1]);
 }
 
-// Butterfly reduce-scatter of N values (N = 8, 16 or 32) over the 32 lanes:
-// on return the lane holds the warp-wide sum of value v = lane >> (5 - log2 N).
-// Each halving step exchanges half of the remaining values with the partner
-// lane (lane ^ o); the lanes left holding the same value after the halving
-// steps are summed by plain butterfly steps.
-template <int N>
+// Butterfly reduce-scatter of N values (N = 8, 16 or 32) over groups of L
+// lanes (L = 16 or 32, aligned): on return the lane holds the group-wide sum of
+// value v = (lane mod L) >> (log2 L - log2 N).  Each halving step exchanges
+// half of the remaining values with the partner lane (lane ^ o); the lanes
+// left holding the same value after the halving steps are summed by plain
+// butterfly steps.
+template <int N, int L>
 __device__ __forceinline__ float reduce_scatter(float (&x)[N], unsigned lane) {
+    static_assert(N <= L, "one value per lane at least");
 #pragma unroll
     for (int st = 0; (N >> st) > 1; ++st) {
-        const int o = 16 >> st;
+        const int o = (L / 2) >> st;
         const int h = (N >> st) / 2;
         const bool upper = (lane & (unsigned)o) != 0;
 #pragma unroll
@@ -168,7 +209,7 @@ __device__ __forceinline__ float reduce_scatter(float (&x)[N], unsigned lane) {
     }
     float s = x[0];
 #pragma unroll
-    for (int o = 16 / N; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    for (int o = L / (2 * N); o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     return s;
 }
 
@@ -229,30 +270,38 @@ decode_partial_kernel(const DecodeArgs a) {
         }
     } else {
         // ---------------------------------------------------------- compute
+        // Lane = (group g, lane-in-group li): group g takes keys
+        // [8w + g*kKPG, 8w + (g+1)*kKPG) of every tile, and li owns head dims
+        // [li*DL, (li+1)*DL) of q, of those keys' K/V rows and of acc.
+        constexpr int LPK = C::LPK;
+        constexpr int DL = C::DL;
+        constexpr int kKPG = C::kKPG;
         const int w = (int)warp;
-        float qr[RMAX][DPL];
+        const int g = (int)(lane / LPK);
+        const int li = (int)(lane % LPK);
+        float qr[RMAX][DL];
         {
             const float qs = a.scale * kLog2e;
-            const T* qg = static_cast<const T*>(a.q) + (size_t)bh * a.R * D + lane * DPL;
+            const T* qg = static_cast<const T*>(a.q) + (size_t)bh * a.R * D + li * DL;
 #pragma unroll
             for (int r = 0; r < RMAX; ++r) {
                 if (r < a.R) {
                     load_row(qg + (size_t)r * D, qr[r]);
 #pragma unroll
-                    for (int i = 0; i < DPL; ++i) qr[r][i] *= qs;
+                    for (int i = 0; i < DL; ++i) qr[r][i] *= qs;
                 } else {
 #pragma unroll
-                    for (int i = 0; i < DPL; ++i) qr[r][i] = 0.f;
+                    for (int i = 0; i < DL; ++i) qr[r][i] = 0.f;
                 }
             }
         }
-        float acc[RMAX][DPL];
+        float acc[RMAX][DL];
 #pragma unroll
         for (int r = 0; r < RMAX; ++r)
 #pragma unroll
-            for (int i = 0; i < DPL; ++i) acc[r][i] = 0.f;
+            for (int i = 0; i < DL; ++i) acc[r][i] = 0.f;
         // this lane's (key, row) value of the reduce-scatter, per pass
-        const int v_mine = (int)(lane >> kSh);
+        const int v_mine = li >> kSh;
         const int j_mine = v_mine / RR;
         float m_mine[C::kPasses], l_mine[C::kPasses];
 #pragma unroll
@@ -264,28 +313,29 @@ decode_partial_kernel(const DecodeArgs a) {
         for (int t = 0; t < n_tiles; ++t) {
             const int s = t % C::kStages;
             if (!mbar_wait(&full[s], (t / C::kStages) & 1, abort_flag)) break;
-            const T* ks = reinterpret_cast<const T*>(smem + (size_t)s * C::kStageBytes) +
-                          (size_t)w * kKeysPerWarp * D + lane * DPL;
+            const int key0 = w * kKeysPerWarp + g * kKPG;            // first key of this group in the tile
+            const T* ks = reinterpret_cast<const T*>(smem + (size_t)s * C::kStageBytes) + (size_t)key0 * D + li * DL;
             const T* vs = ks + C::kTileBytes / (int)sizeof(T);
-            // keys of this warp in this tile that exist (warp-uniform); rows past
-            // it hold stale or unwritten shared memory and are never used
-            const int valid = min(kKeysPerWarp, max(0, n_keys - t * kTK - w * kKeysPerWarp));
-            float kf[kKeysPerWarp][DPL];
-#pragma unroll
-            for (int j = 0; j < kKeysPerWarp; ++j) load_row(ks + j * D, kf[j]);
+            // keys of this group in this tile that exist; rows past them hold
+            // stale or unwritten shared memory and are never used
+            const int valid = min(kKPG, max(0, n_keys - t * kTK - key0));
 #pragma unroll
             for (int p = 0; p < C::kPasses; ++p) {
                 float part[C::kN];
 #pragma unroll
-                for (int j = 0; j < kKeysPerWarp; ++j)
+                for (int j = 0; j < kKPG; ++j) {
+                    float kf[DL];
+                    load_row(ks + j * D, kf);
 #pragma unroll
-                    for (int rr = 0; rr < RR; ++rr) part[j * RR + rr] = dot_slice<DPL>(qr[p * RR + rr], kf[j]);
-                float sv = reduce_scatter<C::kN>(part, lane);
+                    for (int rr = 0; rr < RR; ++rr) part[j * RR + rr] = dot_slice<DL>(qr[p * RR + rr], kf);
+                }
+                float sv = reduce_scatter<C::kN, LPK>(part, lane);
                 sv = (j_mine < valid) ? sv : -INFINITY;
                 float& m = m_mine[p];
                 if (__any_sync(0xffffffffu, sv > m + kRescaleThreshold)) {
                     // exact maximum of this tile per row: over the lanes of the
-                    // same row (the key bits of the value index are lane bits 2-4)
+                    // same row (key bits of the value index: lane bits 2-3 or
+                    // 2-4; group: lane bit 4)
                     float tmax = sv;
 #pragma unroll
                     for (int o = 4; o < 32; o <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
@@ -297,45 +347,57 @@ decode_partial_kernel(const DecodeArgs a) {
                     for (int rr = 0; rr < RR; ++rr) {
                         const float ar = __shfl_sync(0xffffffffu, alpha, rr << kSh);
 #pragma unroll
-                        for (int i = 0; i < DPL; ++i) acc[p * RR + rr][i] *= ar;
+                        for (int i = 0; i < DL; ++i) acc[p * RR + rr][i] *= ar;
                     }
                 }
                 const float pw = (m == -INFINITY) ? 0.f : ex2_approx(sv - m);
                 l_mine[p] += pw;
 #pragma unroll
-                for (int j = 0; j < kKeysPerWarp; ++j) {
+                for (int j = 0; j < kKPG; ++j) {
+                    float vf[DL];
                     if (j < valid) {
-                        float vf[DPL];
                         load_row(vs + j * D, vf);
+                    } else {
 #pragma unroll
-                        for (int rr = 0; rr < RR; ++rr) {
-                            const float pj = __shfl_sync(0xffffffffu, pw, (j * RR + rr) << kSh);
-                            axpy_slice<DPL>(acc[p * RR + rr], pj, vf);
-                        }
+                        for (int i = 0; i < DL; ++i) vf[i] = 0.f;
+                    }
+#pragma unroll
+                    for (int rr = 0; rr < RR; ++rr) {
+                        const float pj = __shfl_sync(0xffffffffu, pw, g * LPK + ((j * RR + rr) << kSh));
+                        axpy_slice<DL>(acc[p * RR + rr], pj, vf);
                     }
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
         }
-        // exp-sum of this warp's keys per row: over the key lanes of each row
+        // exp-sum of this warp's keys per row: over the key lanes and groups of each row
 #pragma unroll
         for (int p = 0; p < C::kPasses; ++p)
 #pragma unroll
             for (int o = 4; o < 32; o <<= 1) l_mine[p] += __shfl_xor_sync(0xffffffffu, l_mine[p], o);
+        // the groups of a warp accumulate the same dims over different keys
+        if constexpr (C::kGroups == 2) {
+#pragma unroll
+            for (int r = 0; r < RMAX; ++r)
+#pragma unroll
+                for (int i = 0; i < DL; ++i) acc[r][i] += __shfl_xor_sync(0xffffffffu, acc[r][i], 16);
+        }
 
         // all compute warps are past the ring before it is reused as scratch
         asm volatile("bar.sync 1, %0;" ::"n"(32 * kCompWarps) : "memory");
         float* sc_acc = reinterpret_cast<float*>(smem);                 // [warp][RMAX][D]
         float* sc_ml = sc_acc + kCompWarps * RMAX * D;                  // [warp][RMAX][2]
+        if (g == 0) {
 #pragma unroll
-        for (int r = 0; r < RMAX; ++r)
+            for (int r = 0; r < RMAX; ++r)
 #pragma unroll
-            for (int i = 0; i < DPL; ++i) sc_acc[(w * RMAX + r) * D + lane * DPL + i] = acc[r][i];
+                for (int i = 0; i < DL; ++i) sc_acc[(w * RMAX + r) * D + li * DL + i] = acc[r][i];
+        }
 #pragma unroll
         for (int p = 0; p < C::kPasses; ++p) {
             // lane (rr << kSh) holds row p*RR + rr (key 0 of the value index)
-            if ((lane & ((1u << kSh) - 1)) == 0 && j_mine == 0) {
+            if (g == 0 && (li & ((1 << kSh) - 1)) == 0 && j_mine == 0) {
                 const int r = p * RR + v_mine;
                 sc_ml[(w * RMAX + r) * 2] = m_mine[p];
                 sc_ml[(w * RMAX + r) * 2 + 1] = l_mine[p];
