@@ -180,22 +180,27 @@ class ClockSampler:
                 "samples": len(rows), "power_w_max": max(power) if power else None}
 
 
-def cpu_oracle_sample(w, seed=0, q_rows=4096):
-    """Time the fp64 oracle's forward + backward on one head, q_rows query rows x all keys."""
-    import numpy as np
+def cpu_oracle_sample(w, seed=0, q_rows=4096, min_seconds=0.0):
+    """Time the fp64 oracle's forward + backward over q_rows query rows x all keys of one head,
+    then of further heads until min_seconds of oracle time have passed (at most all heads)."""
     import oracle
     from synthetic_inputs import to_f64
-    q, k, v, do = make_inputs(custom(1, 1, q_rows, w.Nk, w.D, "bf16", True, name="oracle_sample"), seed)
-    q2, k2, v2, do2 = (to_f64(x)[0, 0] for x in (q, k, v, do))
-    t0 = time.perf_counter()
-    oracle.attention_forward_2d(q2, k2, v2, w.scale)
-    oracle.attention_backward_2d(q2, k2, v2, do2, w.scale)
-    dt = time.perf_counter() - t0
-    flops = 3.5 * 4.0 * q_rows * w.Nk * w.D
+    dt, heads = 0.0, 0
+    while heads < w.B * w.H:
+        q, k, v, do = make_inputs(custom(1, 1, q_rows, w.Nk, w.D, "bf16", True, name="oracle_sample"),
+                                  seed * 1000 + heads)
+        q2, k2, v2, do2 = (to_f64(x)[0, 0] for x in (q, k, v, do))
+        t0 = time.perf_counter()
+        oracle.attention_forward_2d(q2, k2, v2, w.scale)
+        oracle.attention_backward_2d(q2, k2, v2, do2, w.scale)
+        dt += time.perf_counter() - t0
+        heads += 1
+        if dt >= min_seconds:
+            break
+    flops = heads * 3.5 * 4.0 * q_rows * w.Nk * w.D
     cores = len(os.sched_getaffinity(0))
-    del np
-    return flops / dt / 1e12, dt, cores, (f"fp64 numpy oracle, forward then backward of 1 of {w.B * w.H} heads, "
-                                          f"{q_rows} of {w.Nq} query rows x all {w.Nk} keys, D={w.D}")
+    return flops / dt / 1e12, dt, cores, (f"fp64 numpy oracle, forward then backward of {heads} of {w.B * w.H} "
+                                          f"heads, {q_rows} of {w.Nq} query rows x all {w.Nk} keys each, D={w.D}")
 
 
 def run_reference(args):
@@ -557,7 +562,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.no_extras:
-        cv, cdt, cores, sample = cpu_oracle_sample(w)
+        cv, cdt, cores, sample = cpu_oracle_sample(w, min_seconds=10.0)
         cpu = {"value": round(cv, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample,
                "seconds": round(cdt, 2)}
 
