@@ -59,7 +59,9 @@ def test_decode_bf16(B, H, Hkv, Nq, Nk, D):
     (1, 8, 8, 1, 16384, 64),
     (1, 4, 1, 1, 3000, 32),
     (1, 6, 3, 1, 2500, 96),
+    (1, 8, 2, 1, 2000, 96),      # four rows per head at D = 96: half-warps, 6 dims per lane
     (2, 8, 2, 2, 1500, 128),
+    (1, 8, 4, 1, 3000, 128),     # two rows per head, fp32 rows of 512 bytes
     (1, 3, 3, 1, 1, 64),
 ])
 def test_decode_f32(B, H, Hkv, Nq, Nk, D):
