@@ -394,25 +394,40 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tmem_ld32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(&sr[c0]));
                 tmem_wait_ld();
                 const int nvalid = c_end - (c_begin + j * kTileN);
+                // keys past the range get the raw score whose scaled value is -inf
+                const float s_pad = c_log2 >= 0.f ? -INFINITY : INFINITY;
                 if (nvalid < kTileN) {
 #pragma unroll
                     for (int c = 0; c < kTileN; ++c)
-                        if (c >= nvalid) sr[c] = __float_as_uint(-INFINITY);
+                        if (c >= nvalid) sr[c] = __float_as_uint(s_pad);
                 }
-                // row maximum as 8 independent chains of 3-input maxima (one thread
-                // owns the row, so a single 128-long dependent chain would dominate
-                // the softmax latency; the softmax warps are issue-bound, so each
-                // instruction should retire two new values)
-                float mxa[8];
+                // largest scaled score: the raw maximum for scale >= 0, the raw
+                // minimum otherwise; 8 independent chains of 3-input extrema (one
+                // thread owns the row, so a single 128-long dependent chain would
+                // dominate the softmax latency; the softmax warps are issue-bound,
+                // so each instruction should retire two new values)
+                float mx;
+                if (c_log2 >= 0.f) {
+                    float mxa[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) mxa[i] = fmaxf(__uint_as_float(sr[i]), __uint_as_float(sr[8 + i]));
+                    for (int i = 0; i < 8; ++i) mxa[i] = fmaxf(__uint_as_float(sr[i]), __uint_as_float(sr[8 + i]));
 #pragma unroll
-                for (int c = 16; c < kTileN; c += 16)
+                    for (int c = 16; c < kTileN; c += 16)
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        mxa[i] = fmax3(mxa[i], __uint_as_float(sr[c + i]), __uint_as_float(sr[c + 8 + i]));
-                const float mx = fmaxf(fmax3(mxa[0], mxa[1], mxa[2]),
-                                       fmax3(fmax3(mxa[3], mxa[4], mxa[5]), mxa[6], mxa[7]));
+                        for (int i = 0; i < 8; ++i)
+                            mxa[i] = fmax3(mxa[i], __uint_as_float(sr[c + i]), __uint_as_float(sr[c + 8 + i]));
+                    mx = fmaxf(fmax3(mxa[0], mxa[1], mxa[2]), fmax3(fmax3(mxa[3], mxa[4], mxa[5]), mxa[6], mxa[7]));
+                } else {
+                    float mna[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) mna[i] = fminf(__uint_as_float(sr[i]), __uint_as_float(sr[8 + i]));
+#pragma unroll
+                    for (int c = 16; c < kTileN; c += 8)
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) mna[i] = fminf(mna[i], __uint_as_float(sr[c + i]));
+                    mx = fminf(fminf(fminf(mna[0], mna[1]), fminf(mna[2], mna[3])),
+                               fminf(fminf(mna[4], mna[5]), fminf(mna[6], mna[7])));
+                }
                 const float m_blk = mx * c_log2;
                 float m_new = m_ref;
                 bool rescale = false;

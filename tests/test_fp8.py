@@ -81,3 +81,18 @@ def test_fp8_descale_folds_into_scale():
         outs.append((o, lse))
     torch.cuda.synchronize()
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+def test_fp8_negative_scale():
+    """scale < 0: the largest scaled score of a block comes from the smallest raw score."""
+    import exact_memory_efficient_b200 as m
+    w = custom(1, 2, 300, 700, 128, "bf16", backward=False)
+    q8, k8, v, qd, kd = make_inputs_fp8(w, 14)
+    o = torch.empty((1, 2, 300, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((1, 2, 300), dtype=torch.float32, device="cuda")
+    m.mea_attn_fwd_fp8(q8.cuda(), k8.cuda(), v.cuda(), o, lse, -w.scale, qd, kd)
+    assert m.mea_last_device_error() == m.MEA_OK
+    q, k = dequant_f64(q8, qd), dequant_f64(k8, kd)
+    ro, rl = oracle.attention_forward(q, k, to_f64(v), -w.scale)
+    assert_close(to_np(o), ro, *BF16_O, what="fp8 negative scale O")
+    assert_lse_close(to_np(lse), rl, q, k, -w.scale, what="fp8 negative scale lse")

@@ -165,3 +165,52 @@ def test_single_tile_split_repeat(shape):
         assert_close(to_np(dq), rq, *BF16_GRAD, what=f"dQ {shape}", bf16_output=True)
         assert_close(to_np(dk), rk, *BF16_GRAD, what=f"dK {shape}", bf16_output=True)
         assert_close(to_np(dv), rv, *BF16_GRAD, what=f"dV {shape}", bf16_output=True)
+
+
+@pytest.mark.parametrize("B,H,Nq,Nk,D", [
+    (1, 2, 256, 384, 128),    # one CTA per head, three full key tiles
+    (2, 2, 512, 700, 128),    # ragged last key tile: keys 64..127 of it partly missing
+    (1, 3, 768, 65, 128),     # one key tile, one key past its first half
+    (1, 1, 256, 1, 128),      # one key
+    (1, 2, 1024, 1000, 128),  # four CTAs per head
+])
+def test_full_tile_pairs(B, H, Nq, Nk, D):
+    """Nq a multiple of 256 at D = 128: every CTA holds two full query tiles."""
+    w = custom(B, H, Nq, Nk, D, "bf16", backward=False)
+    q, k, v, _ = make_inputs(w, 12)
+    full_check(q, k, v, w.scale, f"tile pairs {(B, H, Nq, Nk, D)}", bf16_output=True)
+
+
+def test_rising_scores_rescale_often():
+    """Scores that grow along the keys make the reference maximum move in most key tiles, so O is
+    rescaled in place many times in both query tiles of every CTA."""
+    Nq, Nk, D = 512, 2048, 128
+    rng = np.random.default_rng(8)
+    q = np.ones((1, 2, Nq, D)) * 0.25 + rng.normal(0, 0.01, (1, 2, Nq, D))
+    ramp = np.linspace(-1.0, 1.0, Nk)[None, None, :, None]
+    k = ramp * 4.0 + rng.normal(0, 0.01, (1, 2, Nk, D))
+    v = rng.normal(0, 1, (1, 2, Nk, D))
+    qt, kt, vt = (torch.tensor(x, dtype=torch.bfloat16) for x in (q, k, v))
+    full_check(qt, kt, vt, 1.0, "rising scores")
+
+
+@pytest.mark.parametrize("B,H,Nq,Nk,D", [
+    (1, 2, 300, 700, 128),    # ragged query tail: the last CTA holds one tile
+    (1, 2, 512, 700, 128),    # full tile pairs
+    (1, 1, 77, 300, 64),
+    (1, 2, 1, 2000, 128),     # decode-shaped: split-KV kernel, scale folded into q
+])
+def test_negative_scale(B, H, Nq, Nk, D):
+    """softmax(scale QK^T) with scale < 0: the block maximum of the scaled scores is the raw minimum."""
+    import exact_memory_efficient_b200 as m
+    w = custom(B, H, Nq, Nk, D, "bf16", backward=True)
+    q, k, v, do = make_inputs(w, 13)
+    scale = -w.scale
+    full_check(q, k, v, scale, f"negative scale {(B, H, Nq, Nk, D)}", bf16_output=True)
+    qd, kd, vd, dod = (x.cuda() for x in (q, k, v, do))
+    o, lse = m.attention_forward(qd, kd, vd, scale)
+    dq, dk, dv = m.attention_backward(qd, kd, vd, o, lse, dod, scale)
+    assert m.mea_last_device_error() == m.MEA_OK
+    rq, rk, rv, _, _ = oracle.attention_backward(to_f64(q), to_f64(k), to_f64(v), to_f64(do), scale)
+    for name, g_, r_ in (("dQ", dq, rq), ("dK", dk, rk), ("dV", dv, rv)):
+        assert_close(to_np(g_), r_, *BF16_GRAD, what=f"negative scale {name}", bf16_output=True)
