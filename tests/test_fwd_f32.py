@@ -85,3 +85,19 @@ def test_deterministic():
     a = run_fwd(q, k, v, w.scale)
     b = run_fwd(q, k, v, w.scale)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("B,H,Nq,Nk,D", [(1, 2, 40, 300, 64), (1, 3, 1, 2000, 128)])
+def test_negative_scale(B, H, Nq, Nk, D):
+    """scale < 0, forward and backward: the SIMT paths scale each score before the running maximum."""
+    import exact_memory_efficient_b200 as m
+    w = custom(B, H, Nq, Nk, D, "f32")
+    q, k, v, do = make_inputs(w, 15)
+    check((q, k, v), -w.scale, "negative scale")
+    qd, kd, vd, dod = (x.cuda() for x in (q, k, v, do))
+    o, lse = m.attention_forward(qd, kd, vd, -w.scale)
+    dq, dk, dv = m.attention_backward(qd, kd, vd, o, lse, dod, -w.scale)
+    assert m.mea_last_device_error() == m.MEA_OK
+    rq, rk, rv, _, _ = oracle.attention_backward(to_f64(q), to_f64(k), to_f64(v), to_f64(do), -w.scale)
+    for name, g_, r_ in (("dQ", dq, rq), ("dK", dk, rk), ("dV", dv, rv)):
+        assert_close(to_np(g_), r_, F32_O_MAX_ABS, what=f"negative scale fp32 {name}")
