@@ -506,6 +506,35 @@ def run_ours(args):
                                   "frac_of_peak": round(wg.bwd_flops() / (b_ms * 1e-3) / 1e12 / peak, 3),
                                   "note": f"mean of {reps}; inputs ({wg.H}+2x{wg.H_kv} heads) fit in L2"}
         del qg, kg, vg, dog, og, lg, wsg, grads
+        # the head-dim-64 configurations (B4 H8 N4096 and B32 H8 N512), forward and
+        # backward through the public API; their inputs fit in L2
+        for wname in ("mha_4k_bf16", "encoder_512_bf16"):
+            wx = make_workload(wname)
+            qx, kx, vx, dox = (x.to(dev) for x in make_inputs(wx, 0))
+            ox, lx = m.attention_forward(qx, kx, vx, wx.scale)
+            wsx = torch.empty(m.mea_attn_bwd_workspace_size(wx.B, wx.H, wx.Nq, wx.Nk, wx.D), dtype=torch.uint8,
+                              device=dev)
+            gx = [torch.empty_like(x) for x in (qx, kx, vx)]
+            for _ in range(3):
+                m.mea_attn_fwd(qx, kx, vx, ox, lx, wx.scale)
+                m.mea_attn_bwd(qx, kx, vx, ox, lx, dox, *gx, wx.scale, wsx)
+            reps = 10
+            ev_x = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+            for e in ev_x:
+                e[0].record(stream)
+                m.mea_attn_fwd(qx, kx, vx, ox, lx, wx.scale)
+                e[1].record(stream)
+                m.mea_attn_bwd(qx, kx, vx, ox, lx, dox, *gx, wx.scale, wsx)
+                e[2].record(stream)
+            torch.cuda.synchronize()
+            f_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev_x)
+            b_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev_x)
+            rows[f"{wname}_fwd"] = {"ms": round(f_ms, 4), "TFLOP/s": round(wx.fwd_flops() / (f_ms * 1e-3) / 1e12, 1),
+                                    "frac_of_peak": round(wx.fwd_flops() / (f_ms * 1e-3) / 1e12 / peak, 3)}
+            rows[f"{wname}_bwd"] = {"ms": round(b_ms, 4), "TFLOP/s": round(wx.bwd_flops() / (b_ms * 1e-3) / 1e12, 1),
+                                    "frac_of_peak": round(wx.bwd_flops() / (b_ms * 1e-3) / 1e12 / peak, 3),
+                                    "note": f"mean of {reps}; D={wx.D}, inputs fit in L2"}
+            del qx, kx, vx, dox, ox, lx, wsx, gx
         # merge of a 4-way key split of the step's workload (HBM-bound): reads four
         # [B,H,N,D] bf16 parts and their lse, writes the merged o and lse
         R = 4
