@@ -25,7 +25,7 @@ BUILD_DIR = os.path.join(PKG_DIR, "_build")
 LIB_NAME = "libmea_attn.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 
-SOURCES = ["api.cu", "fwd_f32.cu", "bwd_f32.cu", "fwd_bf16.cu", "bwd_bf16.cu", "combine.cu", "decode.cu"]
+SOURCES = ["api.cu", "fwd_f32.cu", "bwd_f32.cu", "fwd_bf16.cu", "fwd_persist.cu", "bwd_bf16.cu", "combine.cu", "decode.cu"]
 HEADERS = ["ptx.cuh", "kernels.h", "simt_f32.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -62,6 +62,8 @@ constexpr int kThreads = 320;     // 10 warps
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
+// Bit 13 of a kind::f16 / kind::f8f6f4 instruction descriptor: operand A negated.
+constexpr unsigned kIdescNegateA = 1u << 13;
 
 // F8: Q and K are e4m3 (one byte per element) and S = Q K^T runs as
 // kind::f8f6f4; V, P and O stay bf16.  DEEP: for launches whose CTAs all hold
@@ -216,7 +218,11 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // instructions: descriptors are built once and stepped by 32-bit adds
         // of compile-time offsets; ring stages are tracked incrementally.
         if (lane == 0) {
-            constexpr unsigned idesc_s = make_idesc_bf16(128, kTileN, 0, 0);
+            // scale < 0: S is formed as (-Q) K^T (the instruction's A-negate bit)
+            // and the softmax uses |scale|, so its running maximum is that of the
+            // scaled scores with either sign
+            const unsigned s_neg = scale < 0.f ? kIdescNegateA : 0u;
+            const unsigned idesc_s = make_idesc_bf16(128, kTileN, 0, 0) | s_neg;
             constexpr unsigned idesc_o = make_idesc_bf16(128, D, 0, 1);
             const uint32_t q_lo0 = desc_lo_kmajor(smem_u32(sQ));
             const uint32_t q_lo1 = desc_lo_kmajor(smem_u32(sQ + Cfg::kQBytes));
@@ -238,7 +244,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             auto issue_s = [&](unsigned tS, uint32_t q_lo, uint32_t k_off) {
                 if constexpr (F8) {
                     // K = 32 e4m3 elements per instruction: the same 32-byte step
-                    constexpr unsigned idesc_s8 = make_idesc_e4m3(128, kTileN);
+                    const unsigned idesc_s8 = make_idesc_e4m3(128, kTileN) | s_neg;
 #pragma unroll
                     for (int kk = 0; kk < D / 32; ++kk)
                         mma_ss_lo_f8(tS, q_lo + kmajor_step(kk), ring_k_lo + k_off + kmajor_step(kk), idesc_s8,
@@ -383,7 +389,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 mbar_arrive(&bars->p_ready[t]);
             }
         } else {
-            const float c_log2 = scale * kLog2e;
+            const float c_log2 = fabsf(scale) * kLog2e;   // S carries the sign (A negated)
             for (int it = 0; it < n_mine; ++it) {
                 const int j = split ? 2 * it + t : it;  // key tile within this CTA's range
                 if (!(ok = mbar_wait(&bars->s_full[t], it & 1, abort_flag))) break;
@@ -394,40 +400,25 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tmem_ld32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(&sr[c0]));
                 tmem_wait_ld();
                 const int nvalid = c_end - (c_begin + j * kTileN);
-                // keys past the range get the raw score whose scaled value is -inf
-                const float s_pad = c_log2 >= 0.f ? -INFINITY : INFINITY;
                 if (nvalid < kTileN) {
 #pragma unroll
                     for (int c = 0; c < kTileN; ++c)
-                        if (c >= nvalid) sr[c] = __float_as_uint(s_pad);
+                        if (c >= nvalid) sr[c] = __float_as_uint(-INFINITY);
                 }
-                // largest scaled score: the raw maximum for scale >= 0, the raw
-                // minimum otherwise; 8 independent chains of 3-input extrema (one
-                // thread owns the row, so a single 128-long dependent chain would
-                // dominate the softmax latency; the softmax warps are issue-bound,
-                // so each instruction should retire two new values)
-                float mx;
-                if (c_log2 >= 0.f) {
-                    float mxa[8];
+                // row maximum as 8 independent chains of 3-input maxima (one thread
+                // owns the row, so a single 128-long dependent chain would dominate
+                // the softmax latency; the softmax warps are issue-bound, so each
+                // instruction should retire two new values)
+                float mxa[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) mxa[i] = fmaxf(__uint_as_float(sr[i]), __uint_as_float(sr[8 + i]));
+                for (int i = 0; i < 8; ++i) mxa[i] = fmaxf(__uint_as_float(sr[i]), __uint_as_float(sr[8 + i]));
 #pragma unroll
-                    for (int c = 16; c < kTileN; c += 16)
+                for (int c = 16; c < kTileN; c += 16)
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            mxa[i] = fmax3(mxa[i], __uint_as_float(sr[c + i]), __uint_as_float(sr[c + 8 + i]));
-                    mx = fmaxf(fmax3(mxa[0], mxa[1], mxa[2]), fmax3(fmax3(mxa[3], mxa[4], mxa[5]), mxa[6], mxa[7]));
-                } else {
-                    float mna[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) mna[i] = fminf(__uint_as_float(sr[i]), __uint_as_float(sr[8 + i]));
-#pragma unroll
-                    for (int c = 16; c < kTileN; c += 8)
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) mna[i] = fminf(mna[i], __uint_as_float(sr[c + i]));
-                    mx = fminf(fminf(fminf(mna[0], mna[1]), fminf(mna[2], mna[3])),
-                               fminf(fminf(mna[4], mna[5]), fminf(mna[6], mna[7])));
-                }
+                    for (int i = 0; i < 8; ++i)
+                        mxa[i] = fmax3(mxa[i], __uint_as_float(sr[c + i]), __uint_as_float(sr[c + 8 + i]));
+                const float mx = fmaxf(fmax3(mxa[0], mxa[1], mxa[2]),
+                                       fmax3(fmax3(mxa[3], mxa[4], mxa[5]), mxa[6], mxa[7]));
                 const float m_blk = mx * c_log2;
                 float m_new = m_ref;
                 bool rescale = false;

@@ -96,6 +96,15 @@ struct Bf16FwdArgs {
     bool fp8_qk = false;  // q, k are e4m3 (maps of uint8, box {128, 128, 1}); D = 128 only
 };
 cudaError_t launch_fwd_bf16(const Bf16FwdArgs& a, cudaStream_t stream);
+// The same forward with persistent CTAs (fwd_persist.cu): at most one CTA per
+// SM walks the (head, query-tile pair) items, for bf16 Q/K/V at D = 64 or 128
+// when every item holds two full query tiles (Nq a multiple of 256), the keys
+// are not split and the key range is short: Nk <= 2048 at D = 128, 4096 at
+// D = 64 (longer ranges amortise a CTA's fixed cost by themselves).
+constexpr int kFwdPersistMaxKeys128 = 2048;
+constexpr int kFwdPersistMaxKeys64 = 4096;
+bool fwd_persist_applies(int D, bool fp8_qk, int Nq, int Nk, int chunks);
+cudaError_t launch_fwd_persist(const Bf16FwdArgs& a, int sm_count, cudaStream_t stream);
 // Clusters of `cluster` CTAs of the tensor-core forward instantiation that a
 // launch with these D, operand type and Nq uses that can be resident at once
 // (cudaOccupancyMaxActiveClusters); 0 on failure.

@@ -214,3 +214,19 @@ def test_negative_scale(B, H, Nq, Nk, D):
     rq, rk, rv, _, _ = oracle.attention_backward(to_f64(q), to_f64(k), to_f64(v), to_f64(do), scale)
     for name, g_, r_ in (("dQ", dq, rq), ("dK", dk, rk), ("dV", dv, rv)):
         assert_close(to_np(g_), r_, *BF16_GRAD, what=f"negative scale {name}", bf16_output=True)
+
+
+@pytest.mark.parametrize("B,H,Nq,Nk,D", [
+    (16, 16, 512, 77, 128),   # 512 items over at most one CTA per SM: several items per CTA, one key tile each
+    (8, 16, 256, 200, 64),    # two key tiles, the second ragged
+    (4, 20, 768, 333, 128),   # three query-tile pairs per head, three key tiles
+    (2, 3, 256, 4096, 64),    # the longest key range that takes the persistent CTAs at D = 64
+    (3, 5, 512, 2048, 128),   # and at D = 128
+])
+def test_persistent_items_full(B, H, Nq, Nk, D):
+    """Short key ranges with Nq a multiple of 256: CTAs walk several (head, tile pair) items,
+    reusing their barriers, TMEM and K/V ring from one item to the next."""
+    w = custom(B, H, Nq, Nk, D, "bf16", backward=False)
+    q, k, v, _ = make_inputs(w, 16)
+    full_check(q, k, v, w.scale, f"persistent {(B, H, Nq, Nk, D)}", bf16_output=True)
+    full_check(q, k, v, -w.scale, f"persistent negative scale {(B, H, Nq, Nk, D)}", bf16_output=True)
