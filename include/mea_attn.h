@@ -46,7 +46,11 @@
  *  - Decode-shaped calls (at most 8 query rows per key/value head) over all
  *    SMs with a caller-given workspace: mea_attn_decode.
  *  - Any Nq >= 0 and Nk >= 1; partial tiles are masked.  No mask, no dropout.
- *  - B*H <= 2^31-1 and B*H*max(Nq,Nk)*D < 2^40 elements.
+ *  - B*H*max(Nq,Nk)*D < 2^40 elements, and B*H <= 65535 (one launch-grid
+ *    dimension indexes the heads; the grouped-query entry points count
+ *    B*H_kv).  Decode-shaped calls that the split-KV kernels take accept up
+ *    to 2^31-1 heads.  The fp32 forward also needs ceil(Nq/8) <= 65535.
+ *    Larger calls return MEA_ERR_UNSUPPORTED before any launch.
  */
 #ifndef MEA_ATTN_H
 #define MEA_ATTN_H

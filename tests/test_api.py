@@ -231,3 +231,30 @@ def test_decode_argument_validation(lib):
     assert lib.mea_attn_decode_workspace_size(1, 8, 3, 1, 1024, 128, BF16, ctypes.byref(size)) == 1
     assert lib.mea_attn_decode_workspace_size(1, 8, 8, 1, 1024, 128, BF16, None) == 1
     assert lib.mea_attn_decode_workspace_size(1, 8, 8, 1, 1024, 96, BF16, ctypes.byref(size)) == 2
+
+
+@pytest.mark.gpu
+def test_more_heads_than_the_launch_grid_is_unsupported():
+    """B*H above 65535 (the grid dimension that indexes heads) is refused with
+    MEA_ERR_UNSUPPORTED before any launch.  The tensors are real and sized to
+    the call, so nothing could be read out of bounds even if a kernel ran."""
+    import torch
+    import exact_memory_efficient_b200 as m
+    B, H, N, D = 65536, 1, 16, 64
+    for dt in (torch.bfloat16, torch.float32):
+        q = torch.zeros(B, H, N, D, dtype=dt, device="cuda")
+        o = torch.empty_like(q)
+        lse = torch.empty(B, H, N, device="cuda")
+        with pytest.raises(m.MeaError) as e:
+            m.mea_attn_fwd(q, q, q, o, lse, 0.125)
+        assert e.value.status == 2
+        del q, o, lse
+    q = torch.zeros(B, H, N, D, dtype=torch.bfloat16, device="cuda")
+    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    lse = torch.zeros(B, H, N, device="cuda")
+    ws = torch.empty(m.mea_attn_bwd_workspace_size(B, H, N, N, D), dtype=torch.uint8, device="cuda")
+    with pytest.raises(m.MeaError) as e:
+        m.mea_attn_bwd(q, q, q, o, lse, q, dq, dk, dv, 0.125, ws)
+    assert e.value.status == 2
+    torch.cuda.synchronize()
+    assert m.mea_last_device_error() == 0
