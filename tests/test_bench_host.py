@@ -2,7 +2,9 @@
 
 `roofline.traffic` comes from a committed ncu capture and may only be reported
 while the kernel's own sources are unchanged since that capture; these tests
-pin that rule with a copy of the source tree.
+pin that rule with a copy of the source tree.  The reference arm's JSON line
+(with its oracle sampler stubbed), its rank rule and the warm-up minimum are
+checked too.
 """
 
 import importlib.util
@@ -57,3 +59,48 @@ def test_committed_traffic_names_known_kernels():
     for name, e in d.items():
         assert name.split("<")[0] in b.KERNEL_SOURCES, name
         assert e["dram_bytes_per_launch"] == int(e["dram_read"] + e["dram_write"]), name
+
+
+def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
+    """`--impl reference` prints one JSON line with the keys of the bench
+    contract; the oracle sampler is replaced by a stub so no oracle work runs."""
+    import argparse
+    bench = _load_bench(ROOT)
+    calls = []
+
+    def fake_sample(w, seed):
+        calls.append(seed)
+        return 0.02 + 0.001 * len(calls), 1.5, 8, "stub sample"
+
+    monkeypatch.setattr(bench, "cpu_oracle_sample", fake_sample)
+    monkeypatch.delenv("RANK", raising=False)
+    assert bench.run_reference(argparse.Namespace(gpus=1, steps=2, warmup=3)) == 0
+    assert len(calls) == 5                        # warm-up samples run too, and are discarded
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["value"] == round((0.024 + 0.025) / 2, 6)   # median of the two timed samples
+    assert line["config"]["workload"] == bench.WORKLOAD
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 8
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_without_work(monkeypatch, capsys):
+    import argparse
+    bench = _load_bench(ROOT)
+    monkeypatch.setattr(bench, "cpu_oracle_sample", lambda w, seed: (_ for _ in ()).throw(AssertionError))
+    monkeypatch.setenv("RANK", "1")
+    assert bench.run_reference(argparse.Namespace(gpus=2, steps=2, warmup=3)) == 0
+    assert capsys.readouterr().out == ""
+
+
+def test_fewer_than_three_warmup_steps_is_refused(monkeypatch):
+    import pytest
+    bench = _load_bench(ROOT)
+    monkeypatch.setattr("sys.argv", ["bench.py", "--warmup", "2"])
+    with pytest.raises(SystemExit) as e:
+        bench.main()
+    assert e.value.code == 2
