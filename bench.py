@@ -642,7 +642,7 @@ def run_profile(name: str) -> int:
     return 0
 
 
-def main():
+def build_parser() -> argparse.ArgumentParser:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -657,6 +657,11 @@ def main():
     ap.add_argument("--profile", metavar="WORKLOAD", default=None,
                     help="no timing: run this workload's forward (and backward, if it has one) three times and "
                          "exit; the command profiling captures wrap (forward-only workloads: mea_attn_decode)")
+    return ap
+
+
+def main():
+    ap = build_parser()
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

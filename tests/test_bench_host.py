@@ -4,7 +4,7 @@
 while the kernel's own sources are unchanged since that capture; these tests
 pin that rule with a copy of the source tree.  The reference arm's JSON line
 (with its oracle sampler stubbed), its rank rule and the warm-up minimum are
-checked too.
+checked too, and every bench command recorded in profiles/ must still parse.
 """
 
 import importlib.util
@@ -104,3 +104,25 @@ def test_fewer_than_three_warmup_steps_is_refused(monkeypatch):
     with pytest.raises(SystemExit) as e:
         bench.main()
     assert e.value.code == 2
+
+
+def test_profile_commands_parse_with_the_current_bench():
+    """Every `python bench.py ...` command recorded in profiles/*.md is accepted
+    by the current argument parser, and names a known workload."""
+    import glob
+    import re
+    import shlex
+    from synthetic_inputs import WORKLOADS
+    bench = _load_bench(ROOT)
+    found = 0
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        for line in open(path, encoding="utf-8"):
+            m = re.search(r"python bench\.py((?:\s+--?[\w-]+(?:\s+[\w.]+)?)*)", line)
+            if not m:
+                continue
+            args = bench.build_parser().parse_args(shlex.split(m.group(1)))
+            assert args.warmup >= 3, (path, line)
+            for name in (args.workload, args.profile):
+                assert name is None or name in WORKLOADS, (path, name)
+            found += 1
+    assert found >= 4
