@@ -5,11 +5,17 @@ Tolerances
 * bf16 paths: O within max-abs 2e-2 and relative Frobenius 5e-3 of the fp64
   oracle; dQ, dK, dV within max-abs 3e-2 and relative Frobenius 1e-2.
 * fp32 path: O within max-abs 1e-4.
-* The stated absolute bounds presume outputs of order one (N(0,1) inputs).
-  Edge cases that produce larger outputs (a single key, so that dV sums every
-  dO row) are checked with the bound widened by the bf16 rounding of the
-  stored output itself: max_abs_tol + 2^-8 |ref| per element (a bf16 result
-  carries up to 2^-9 relative rounding error before any arithmetic error).
+* The stated absolute bounds presume outputs of order one (N(0,1) inputs,
+  |ref| <= ORDER_ONE = 4), and every order-one tensor is held to them.  Only a
+  construction that makes a tensor large -- few keys shared by many query
+  rows, so that dV and dK sum many rows (a single key: dV_0 = sum_i dO_i,
+  |dV| ~ 30-80) -- may pass ``large_outputs=True``.  The helper then asserts
+  that the reference really exceeds ORDER_ONE, and scales the absolute bound
+  of that tensor by max|ref| / ORDER_ONE: the rounding errors of these sums
+  (bf16 P and dS, half an ulp of bf16 being 2^-9 relative) grow with the
+  magnitude of the summed terms, which is that of the largest outputs, and
+  half an ulp of a bf16 value of 8 (2^-5) already exceeds 3e-2.  The relative
+  Frobenius bound is never widened.
 * lse (no tolerance is stated for it; derived from the arithmetic): the
   kernels evaluate lse_i = m_i + ln l_i in fp32 from scores s_ij = scale * q_i.k_j
   accumulated in fp32 and from Nk exponentials summed in fp32.  The error is
@@ -30,6 +36,7 @@ U32 = 2.0 ** -24
 BF16_O = (2e-2, 5e-3)
 BF16_GRAD = (3e-2, 1e-2)
 F32_O_MAX_ABS = 1e-4
+ORDER_ONE = 4.0
 
 
 def errors(gpu, ref):
@@ -45,15 +52,16 @@ def errors(gpu, ref):
     return max_abs, rel
 
 
-def assert_close(gpu, ref, max_abs_tol, rel_tol=None, what="", bf16_output=False):
+def assert_close(gpu, ref, max_abs_tol, rel_tol=None, what="", large_outputs=False):
     ma, rf = errors(gpu, ref)
     g = np.asarray(gpu, dtype=np.float64)
     assert np.isfinite(g).all(), f"{what}: non-finite values"
-    if bf16_output:
-        r = np.asarray(ref, dtype=np.float64)
-        excess = np.abs(g - r) - (max_abs_tol + 2.0 ** -8 * np.abs(r))
-        assert (excess <= 0).all(), f"{what}: {int((excess > 0).sum())} elements beyond max-abs " \
-                                    f"{max_abs_tol:.1e} + 2^-8|ref| (max-abs {ma:.3e})"
+    if large_outputs:
+        top = float(np.abs(np.asarray(ref, dtype=np.float64)).max())
+        assert top > ORDER_ONE, f"{what}: large_outputs given for an order-one reference (max |ref| {top:.2f})"
+        bound = max_abs_tol * top / ORDER_ONE
+        assert ma <= bound, f"{what}: max-abs {ma:.3e} > {bound:.3e} ({max_abs_tol:.1e} x max|ref| {top:.1f} / " \
+                            f"{ORDER_ONE}) (rel-Frob {rf:.3e})"
     else:
         assert ma <= max_abs_tol, f"{what}: max-abs {ma:.3e} > {max_abs_tol:.1e} (rel-Frob {rf:.3e})"
     if rel_tol is not None:

@@ -39,9 +39,10 @@ def test_shapes_full(B, H, Nq, Nk, D):
     dq, dk, dv = gpu_fwd_bwd(q, k, v, do, w.scale)
     rq, rk, rv, _, _ = oracle.attention_backward(to_f64(q), to_f64(k), to_f64(v), to_f64(do), w.scale)
     what = f"{(B, H, Nq, Nk, D)}"
-    assert_close(to_np(dq), rq, *BF16_GRAD, what=f"dQ {what}", bf16_output=True)
-    assert_close(to_np(dk), rk, *BF16_GRAD, what=f"dK {what}", bf16_output=True)
-    assert_close(to_np(dv), rv, *BF16_GRAD, what=f"dV {what}", bf16_output=True)
+    assert_close(to_np(dq), rq, *BF16_GRAD, what=f"dQ {what}")
+    assert_close(to_np(dk), rk, *BF16_GRAD, what=f"dK {what}")
+    # a single key makes dV_0 the sum of every dO row (|dV| ~ 33 here): beyond order one
+    assert_close(to_np(dv), rv, *BF16_GRAD, what=f"dV {what}", large_outputs=(Nk == 1))
 
 
 @pytest.mark.parametrize("seed", [0, 1, 2])

@@ -26,11 +26,11 @@ def gpu_fwd(q, k, v, scale):
     return o, lse
 
 
-def full_check(q, k, v, scale, what, bf16_output=False):
+def full_check(q, k, v, scale, what):
     o, lse = gpu_fwd(q, k, v, scale)
     q64, k64, v64 = to_f64(q), to_f64(k), to_f64(v)
     o_ref, lse_ref = oracle.attention_forward(q64, k64, v64, scale)
-    assert_close(to_np(o), o_ref, *BF16_O, what=f"O {what}", bf16_output=bf16_output)
+    assert_close(to_np(o), o_ref, *BF16_O, what=f"O {what}")
     assert_lse_close(to_np(lse), lse_ref, q64, k64, scale, what=f"lse {what}")
 
 
@@ -47,7 +47,7 @@ def full_check(q, k, v, scale, what, bf16_output=False):
 def test_shapes_full(B, H, Nq, Nk, D):
     w = custom(B, H, Nq, Nk, D, "bf16", backward=False)
     q, k, v, _ = make_inputs(w, 11)
-    full_check(q, k, v, w.scale, f"{(B, H, Nq, Nk, D)}", bf16_output=True)
+    full_check(q, k, v, w.scale, f"{(B, H, Nq, Nk, D)}")
 
 
 @pytest.mark.parametrize("B,H,Nq,Nk,D", [
@@ -60,7 +60,7 @@ def test_shapes_full(B, H, Nq, Nk, D):
 def test_decode_key_split(B, H, Nq, Nk, D):
     w = custom(B, H, Nq, Nk, D, "bf16", backward=False)
     q, k, v, _ = make_inputs(w, 17)
-    full_check(q, k, v, w.scale, f"{(B, H, Nq, Nk, D)}", bf16_output=True)
+    full_check(q, k, v, w.scale, f"{(B, H, Nq, Nk, D)}")
 
 
 @pytest.mark.parametrize("seed", [0, 1, 2])
@@ -162,9 +162,9 @@ def test_single_tile_split_repeat(shape):
         assert m.mea_last_device_error() == m.MEA_OK
         assert_close(to_np(o), ro, *BF16_O, what=f"O {shape}")
         assert_lse_close(to_np(lse), rl, to_f64(q), to_f64(k), w.scale, what=f"lse {shape}")
-        assert_close(to_np(dq), rq, *BF16_GRAD, what=f"dQ {shape}", bf16_output=True)
-        assert_close(to_np(dk), rk, *BF16_GRAD, what=f"dK {shape}", bf16_output=True)
-        assert_close(to_np(dv), rv, *BF16_GRAD, what=f"dV {shape}", bf16_output=True)
+        assert_close(to_np(dq), rq, *BF16_GRAD, what=f"dQ {shape}")
+        assert_close(to_np(dk), rk, *BF16_GRAD, what=f"dK {shape}")
+        assert_close(to_np(dv), rv, *BF16_GRAD, what=f"dV {shape}")
 
 
 @pytest.mark.parametrize("B,H,Nq,Nk,D", [
@@ -178,7 +178,7 @@ def test_full_tile_pairs(B, H, Nq, Nk, D):
     """Nq a multiple of 256 at D = 128: every CTA holds two full query tiles."""
     w = custom(B, H, Nq, Nk, D, "bf16", backward=False)
     q, k, v, _ = make_inputs(w, 12)
-    full_check(q, k, v, w.scale, f"tile pairs {(B, H, Nq, Nk, D)}", bf16_output=True)
+    full_check(q, k, v, w.scale, f"tile pairs {(B, H, Nq, Nk, D)}")
 
 
 def test_rising_scores_rescale_often():
@@ -206,14 +206,14 @@ def test_negative_scale(B, H, Nq, Nk, D):
     w = custom(B, H, Nq, Nk, D, "bf16", backward=True)
     q, k, v, do = make_inputs(w, 13)
     scale = -w.scale
-    full_check(q, k, v, scale, f"negative scale {(B, H, Nq, Nk, D)}", bf16_output=True)
+    full_check(q, k, v, scale, f"negative scale {(B, H, Nq, Nk, D)}")
     qd, kd, vd, dod = (x.cuda() for x in (q, k, v, do))
     o, lse = m.attention_forward(qd, kd, vd, scale)
     dq, dk, dv = m.attention_backward(qd, kd, vd, o, lse, dod, scale)
     assert m.mea_last_device_error() == m.MEA_OK
     rq, rk, rv, _, _ = oracle.attention_backward(to_f64(q), to_f64(k), to_f64(v), to_f64(do), scale)
     for name, g_, r_ in (("dQ", dq, rq), ("dK", dk, rk), ("dV", dv, rv)):
-        assert_close(to_np(g_), r_, *BF16_GRAD, what=f"negative scale {name}", bf16_output=True)
+        assert_close(to_np(g_), r_, *BF16_GRAD, what=f"negative scale {name}")
 
 
 @pytest.mark.parametrize("B,H,Nq,Nk,D", [
@@ -228,5 +228,5 @@ def test_persistent_items_full(B, H, Nq, Nk, D):
     reusing their barriers, TMEM and K/V ring from one item to the next."""
     w = custom(B, H, Nq, Nk, D, "bf16", backward=False)
     q, k, v, _ = make_inputs(w, 16)
-    full_check(q, k, v, w.scale, f"persistent {(B, H, Nq, Nk, D)}", bf16_output=True)
-    full_check(q, k, v, -w.scale, f"persistent negative scale {(B, H, Nq, Nk, D)}", bf16_output=True)
+    full_check(q, k, v, w.scale, f"persistent {(B, H, Nq, Nk, D)}")
+    full_check(q, k, v, -w.scale, f"persistent negative scale {(B, H, Nq, Nk, D)}")

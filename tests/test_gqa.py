@@ -41,9 +41,10 @@ def test_gqa_bf16_forward_backward(B, H, Hkv, Nq, Nk, D):
     assert_close(to_np(o), ro, *BF16_O, what=f"O {what}")
     assert_lse_close(to_np(lse), rl, to_f64(q), np.repeat(to_f64(k), H // Hkv, axis=1), w.scale,
                      what=f"lse {what}")
-    assert_close(to_np(dq), rq, *BF16_GRAD, what=f"dQ {what}", bf16_output=True)
-    assert_close(to_np(dk), rk, *BF16_GRAD, what=f"dK {what}", bf16_output=True)
-    assert_close(to_np(dv), rv, *BF16_GRAD, what=f"dV {what}", bf16_output=True)
+    assert_close(to_np(dq), rq, *BF16_GRAD, what=f"dQ {what}")
+    assert_close(to_np(dk), rk, *BF16_GRAD, what=f"dK {what}")
+    # a single key makes dV the sum of every dO row of the group (|dV| ~ 80 here): beyond order one
+    assert_close(to_np(dv), rv, *BF16_GRAD, what=f"dV {what}", large_outputs=(Nk == 1))
 
 
 def test_gqa_equal_heads_is_the_per_head_path():
@@ -133,5 +134,5 @@ def test_gqa_workload_sampled(seed):
             dk_h, dv_h = oracle.attention_backward_keys(q2, k2, v2, do2, w.scale, keys, lse_all, o_all)
             rk += dk_h
             rv += dv_h
-        assert_close(dk[0, hk][keys], rk, *BF16_GRAD, what=f"dK kv head {hk}", bf16_output=True)
-        assert_close(dv[0, hk][keys], rv, *BF16_GRAD, what=f"dV kv head {hk}", bf16_output=True)
+        assert_close(dk[0, hk][keys], rk, *BF16_GRAD, what=f"dK kv head {hk}")
+        assert_close(dv[0, hk][keys], rv, *BF16_GRAD, what=f"dV kv head {hk}")

@@ -38,14 +38,24 @@ def test_assert_close_applies_both_bounds():
         assert_close(np.array([np.nan, 1.0]), np.array([1.0, 1.0]), 1.0)
 
 
-def test_bf16_output_widening():
+def test_large_output_widening():
     ref = np.array([32.0, 1.0])
-    # 32 + 0.1: beyond 2e-2 plain, inside 2e-2 + 2^-8 * 32 = 0.145
-    assert_close(ref + np.array([0.1, 0.0]), ref, 2e-2, bf16_output=True)
+    # max|ref| = 32: the absolute bound 2e-2 scales to 2e-2 * 32 / 4 = 0.16, on every element
+    assert_close(ref + np.array([0.15, 0.0]), ref, 2e-2, large_outputs=True)
+    assert_close(ref + np.array([0.0, 0.15]), ref, 2e-2, large_outputs=True)
     with pytest.raises(AssertionError):
         assert_close(ref + np.array([0.1, 0.0]), ref, 2e-2)
     with pytest.raises(AssertionError):
-        assert_close(ref + np.array([0.2, 0.0]), ref, 2e-2, bf16_output=True)
+        assert_close(ref + np.array([0.17, 0.0]), ref, 2e-2, large_outputs=True)
+    # the relative Frobenius bound is not widened
+    with pytest.raises(AssertionError):
+        assert_close(ref + np.array([0.15, 0.15]), ref, 2e-2, 1e-3, large_outputs=True)
+
+
+def test_large_output_flag_refused_on_order_one_reference():
+    ref = np.array([3.9, -1.0])
+    with pytest.raises(AssertionError, match="order-one"):
+        assert_close(ref, ref, 2e-2, large_outputs=True)
 
 
 def _lse_fp32(q, k, scale):
