@@ -26,7 +26,7 @@ __all__ = [
     "MeaError", "load_library", "library_path",
     "MEA_OK", "MEA_ERR_INVALID_ARG", "MEA_ERR_UNSUPPORTED", "MEA_ERR_MISALIGNED", "MEA_ERR_WORKSPACE",
     "MEA_ERR_CUDA", "MEA_ERR_TIMEOUT", "MEA_DTYPE_F32", "MEA_DTYPE_BF16",
-    "MEA_BWD_ALL", "MEA_BWD_PREPROCESS", "MEA_BWD_MAIN", "MEA_BWD_FINALIZE",
+    "MEA_BWD_ALL", "MEA_BWD_PREPROCESS", "MEA_BWD_MAIN", "MEA_BWD_FINALIZE", "MEA_NOALLOC_SCRATCH_BYTES",
     "mea_attn_fwd", "mea_attn_bwd", "mea_attn_bwd_phase", "mea_attn_bwd_workspace_size", "mea_attn_bwd_noalloc",
     "mea_attn_fwd_gqa", "mea_attn_bwd_gqa", "mea_attn_bwd_gqa_workspace_size", "mea_attn_fwd_fp8",
     "mea_attn_combine", "mea_attn_decode", "mea_attn_decode_workspace_size", "attention_decode",
@@ -49,6 +49,9 @@ MEA_BWD_ALL = 0
 MEA_BWD_PREPROCESS = 1
 MEA_BWD_MAIN = 2
 MEA_BWD_FINALIZE = 3
+
+# size of the static device scratch behind mea_attn_bwd_noalloc (include/mea_attn.h)
+MEA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -161,6 +164,41 @@ def _bhnd(t: torch.Tensor, name: str):
     return t.shape
 
 
+def _shape4(t, name: str):
+    if t is None or t.dim() != 4:
+        raise MeaError(MEA_ERR_INVALID_ARG, f"{name} must be [B, H, N, D]")
+    return tuple(t.shape)
+
+
+def _bwd_operands(q, k, v, o, lse, do, dq, dk, dv, where: str) -> None:
+    """o, do, dq shaped like q; v, dk, dv like k; one dtype; lse fp32 [B, H, Nq]; then all
+    contiguous CUDA tensors.  Checked before any launch, since the kernels index every operand
+    by q's and k's sizes."""
+    qs, ks = _shape4(q, "q"), _shape4(k, "k")
+    for name, t, shape in (("o", o, qs), ("do", do, qs), ("dq", dq, qs), ("v", v, ks), ("dk", dk, ks),
+                           ("dv", dv, ks)):
+        if _shape4(t, name) != shape or t.dtype != q.dtype:
+            raise MeaError(MEA_ERR_INVALID_ARG, f"{where}: {name} shape/dtype mismatch")
+    if k.dtype != q.dtype:
+        raise MeaError(MEA_ERR_INVALID_ARG, f"{where}: k dtype mismatch")
+    if lse is None or tuple(lse.shape) != qs[:3] or lse.dtype != torch.float32:
+        raise MeaError(MEA_ERR_INVALID_ARG, f"{where}: lse must be fp32 [B, H, Nq]")
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do), ("dq", dq), ("dk", dk), ("dv", dv),
+                    ("lse", lse)):
+        if not t.is_contiguous() or not t.is_cuda:
+            raise MeaError(MEA_ERR_INVALID_ARG, f"{where}: {name} must be a contiguous CUDA tensor")
+
+
+def _bwd_shapes(q, k, v, o, lse, do, dq, dk, dv, where: str):
+    """Shapes of a backward with one key/value head per query head: k [B, H, Nk, D] with q's B, H, D."""
+    B, H, Nq, D = _shape4(q, "q")
+    Bk, Hk, Nk, Dk = _shape4(k, "k")
+    if (Bk, Hk, Dk) != (B, H, D):
+        raise MeaError(MEA_ERR_INVALID_ARG, f"{where}: k must be [B, H, Nk, D] with q's B, H and D")
+    _bwd_operands(q, k, v, o, lse, do, dq, dk, dv, where)
+    return B, H, Nq, Nk, D
+
+
 def mea_attn_fwd(q, k, v, o, lse, scale: float, stream=None) -> None:
     """C ``mea_attn_fwd``: writes o [B,H,Nq,D] and lse [B,H,Nq] (fp32) on the stream."""
     B, H, Nq, D = _bhnd(q, "q")
@@ -191,12 +229,7 @@ def mea_attn_bwd(q, k, v, o, lse, do, dq, dk, dv, scale: float, workspace, strea
 
 def mea_attn_bwd_phase(phase: int, q, k, v, o, lse, do, dq, dk, dv, scale: float, workspace, stream=None) -> None:
     """C ``mea_attn_bwd_phase``: one phase (MEA_BWD_*) of the backward pass."""
-    B, H, Nq, D = _bhnd(q, "q")
-    _, _, Nk, _ = _bhnd(k, "k")
-    for name, t, shape in (("o", o, q.shape), ("do", do, q.shape), ("dq", dq, q.shape), ("v", v, k.shape),
-                           ("dk", dk, k.shape), ("dv", dv, k.shape)):
-        if tuple(t.shape) != tuple(shape) or t.dtype != q.dtype:
-            raise MeaError(MEA_ERR_INVALID_ARG, f"mea_attn_bwd: {name} shape/dtype mismatch")
+    B, H, Nq, Nk, D = _bwd_shapes(q, k, v, o, lse, do, dq, dk, dv, "mea_attn_bwd")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = load_library().mea_attn_bwd_phase(int(phase), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do),
                                             _ptr(dq), _ptr(dk), _ptr(dv), B, H, Nq, Nk, D, float(scale),
@@ -207,23 +240,21 @@ def mea_attn_bwd_phase(phase: int, q, k, v, o, lse, do, dq, dk, dv, scale: float
 def mea_attn_bwd_noalloc(q, k, v, o, lse, do, dq, dk, dv, scale: float, stream=None) -> None:
     """C ``mea_attn_bwd_noalloc``: the backward with the library's static scratch instead of a
     caller workspace (for callers that cannot allocate; sizes up to a 64 MiB workspace)."""
-    B, H, Nq, D = _bhnd(q, "q")
-    _, _, Nk, _ = _bhnd(k, "k")
-    for name, t, shape in (("o", o, q.shape), ("do", do, q.shape), ("dq", dq, q.shape), ("v", v, k.shape),
-                           ("dk", dk, k.shape), ("dv", dv, k.shape)):
-        if tuple(t.shape) != tuple(shape) or t.dtype != q.dtype:
-            raise MeaError(MEA_ERR_INVALID_ARG, f"mea_attn_bwd_noalloc: {name} shape/dtype mismatch")
+    B, H, Nq, Nk, D = _bwd_shapes(q, k, v, o, lse, do, dq, dk, dv, "mea_attn_bwd_noalloc")
     st = load_library().mea_attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq),
                                               _ptr(dk), _ptr(dv), B, H, Nq, Nk, D, float(scale), _dtype_code(q),
                                               _stream_handle(stream))
     _check(st, "mea_attn_bwd_noalloc")
 
 
-def _gqa_shapes(q, k, where: str):
-    B, H, Nq, D = _bhnd(q, "q")
-    Bk, Hkv, Nk, Dk = _bhnd(k, "k")
+def _gqa_shapes(q, k, where: str, check_device: bool = True):
+    B, H, Nq, D = _shape4(q, "q")
+    Bk, Hkv, Nk, Dk = _shape4(k, "k")
     if (Bk, Dk) != (B, D) or Hkv < 1 or H % Hkv != 0:
         raise MeaError(MEA_ERR_INVALID_ARG, f"{where}: k must be [B, H_kv, Nk, D] with H a multiple of H_kv")
+    if check_device:
+        _bhnd(q, "q")
+        _bhnd(k, "k")
     return B, H, Hkv, Nq, Nk, D
 
 
@@ -253,11 +284,8 @@ def mea_attn_bwd_gqa_workspace_size(B: int, H: int, H_kv: int, Nq: int, Nk: int,
 
 def mea_attn_bwd_gqa(q, k, v, o, lse, do, dq, dk, dv, scale: float, workspace, stream=None) -> None:
     """C ``mea_attn_bwd_gqa``: dq [B,H,Nq,D]; dk, dv [B,H_kv,Nk,D] summed over each group."""
-    B, H, Hkv, Nq, Nk, D = _gqa_shapes(q, k, "mea_attn_bwd_gqa")
-    for name, t, shape in (("o", o, q.shape), ("do", do, q.shape), ("dq", dq, q.shape), ("v", v, k.shape),
-                           ("dk", dk, k.shape), ("dv", dv, k.shape)):
-        if tuple(t.shape) != tuple(shape) or t.dtype != q.dtype:
-            raise MeaError(MEA_ERR_INVALID_ARG, f"mea_attn_bwd_gqa: {name} shape/dtype mismatch")
+    B, H, Hkv, Nq, Nk, D = _gqa_shapes(q, k, "mea_attn_bwd_gqa", check_device=False)  # device checked below
+    _bwd_operands(q, k, v, o, lse, do, dq, dk, dv, "mea_attn_bwd_gqa")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = load_library().mea_attn_bwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq),
                                           _ptr(dk), _ptr(dv), B, H, Hkv, Nq, Nk, D, float(scale), _dtype_code(q),

@@ -622,8 +622,41 @@ mea_status_t mea_attn_bwd_gqa(const void* q, const void* k, const void* v, const
 namespace {
 constexpr size_t kNoAllocScratchBytes = (size_t)MEA_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
-void* g_noalloc_ptr[kMaxDevices] = {};
+// The array's device address, resolved once per device and remembered with
+// the unique id of the context it was resolved in: a device reset (or any new
+// context) loads the module again, possibly elsewhere, so a changed id means
+// the address is resolved anew instead of handing a freed address to a kernel.
+struct NoAllocScratch {
+    void* ptr = nullptr;
+    unsigned long long ctx_id = 0;
+};
+NoAllocScratch g_noalloc[kMaxDevices];
 std::mutex g_noalloc_mu;
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+
+// Id of the context current on this thread, 0 if none is current yet.
+mea_status_t current_context_id(unsigned long long* id) {
+    *id = 0;
+    if (g_ctx_get_current == nullptr || g_ctx_get_id == nullptr) {
+        void* f1 = nullptr;
+        void* f2 = nullptr;
+        cudaDriverEntryPointQueryResult q1, q2;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+            q1 != cudaDriverEntryPointSuccess || f1 == nullptr ||
+            cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+            q2 != cudaDriverEntryPointSuccess || f2 == nullptr)
+            return fail(MEA_ERR_CUDA, "cudaGetDriverEntryPoint", "cuCtxGetCurrent/cuCtxGetId unavailable");
+        g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+        g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(f2);
+    }
+    CUcontext ctx = nullptr;
+    if (g_ctx_get_current(&ctx) != CUDA_SUCCESS) return fail(MEA_ERR_CUDA, "cuCtxGetCurrent", "failed");
+    if (ctx != nullptr && g_ctx_get_id(ctx, id) != CUDA_SUCCESS) return fail(MEA_ERR_CUDA, "cuCtxGetId", "failed");
+    return MEA_OK;
+}
 }  // namespace
 
 extern "C" {
@@ -648,16 +681,22 @@ mea_status_t mea_attn_bwd_noalloc(const void* q, const void* k, const void* v, c
     if (dev < 0 || dev >= kMaxDevices) return MEA_ERR_UNSUPPORTED;
     void* scratch = nullptr;
     {
-        // One-time set-up per device, with that device current: resolve the
-        // device address of the static scratch array.
+        // Set-up once per device (and again only if the device's context was
+        // replaced), with that device current: resolve the device address of
+        // the static scratch array.  Host code never passes the array's name.
         std::lock_guard<std::mutex> lk(g_noalloc_mu);
-        if (g_noalloc_ptr[dev] == nullptr) {
+        unsigned long long ctx_id = 0;
+        if ((st = current_context_id(&ctx_id)) != MEA_OK) return st;
+        NoAllocScratch& s = g_noalloc[dev];
+        if (s.ptr == nullptr || ctx_id == 0 || ctx_id != s.ctx_id) {
             void* p = nullptr;
-            e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+            e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // also makes the device's context current
             if (e != cudaSuccess || p == nullptr) return fail_cuda("cudaGetSymbolAddress(scratch)", e);
-            g_noalloc_ptr[dev] = p;
+            if ((st = current_context_id(&ctx_id)) != MEA_OK) return st;
+            s.ptr = p;
+            s.ctx_id = ctx_id;
         }
-        scratch = g_noalloc_ptr[dev];
+        scratch = s.ptr;
     }
     // The preprocess phase re-zeroes the dQ accumulator and rewrites the row
     // term on every call, so nothing left by an earlier call is read.

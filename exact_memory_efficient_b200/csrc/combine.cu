@@ -74,6 +74,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
 #pragma unroll
     for (int r = 0; r < MAXR; ++r)
         if (r < a.R) load8(static_cast<const T*>(a.o_parts[r]) + row * a.D + 8 * g, x[r]);
+    // a row whose parts are all empty has no keys at all: its sum of exponentials
+    // is 0, so lse = ln 0 = -inf, and its o is written as 0 (every weight is 0)
+    const bool no_keys = (M == -INFINITY);
+    const float Mref = no_keys ? 0.f : M;
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
@@ -81,18 +85,18 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
 #pragma unroll
     for (int r = 0; r < MAXR; ++r) {
         if (r < a.R) {
-            const float w = ex2_approx((lv[r] - M) * kLog2e);
+            const float w = ex2_approx((lv[r] - Mref) * kLog2e);
             const bool use = w != 0.f;
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc[i] = use ? fmaf(w, x[r][i], acc[i]) : acc[i];
             L += w;
         }
     }
-    const float inv = 1.f / L;
+    const float inv = no_keys ? 0.f : 1.f / L;
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] *= inv;
     store8(static_cast<T*>(a.o) + row * a.D + 8 * g, acc);
-    if (g == 0) a.lse[row] = M + __log2f(L) * kLn2;
+    if (g == 0) a.lse[row] = no_keys ? -INFINITY : M + __log2f(L) * kLn2;
 }
 
 }  // namespace

@@ -46,10 +46,12 @@ class CudaOps:
         """PREPROCESS + MAIN over this rank's keys; returns (fp32 dQ accumulator, dk, dv, finish)."""
         m = self.m
         B, H, Nq, D = q.shape
-        ws = torch.empty(m.mea_attn_bwd_workspace_size(B, H, Nq, k.shape[2], D, q.dtype), dtype=torch.uint8,
-                         device=q.device)
         dq = torch.empty_like(q)
         dk, dv = torch.empty_like(k), torch.empty_like(v)
+        if k.shape[2] == 0:
+            return self._backward_no_keys(q, o, lse, do, dq, dk, dv, scale)
+        ws = torch.empty(m.mea_attn_bwd_workspace_size(B, H, Nq, k.shape[2], D, q.dtype), dtype=torch.uint8,
+                         device=q.device)
         for ph in (m.MEA_BWD_PREPROCESS, m.MEA_BWD_MAIN):
             m.mea_attn_bwd_phase(ph, q, k, v, o, lse, do, dq, dk, dv, scale, ws)
         if q.dtype == torch.float32:
@@ -60,6 +62,26 @@ class CudaOps:
         def finish(summed):
             # FINALIZE reads the (now summed) accumulator in place
             m.mea_attn_bwd_phase(m.MEA_BWD_FINALIZE, q, k, v, o, lse, do, dq, dk, dv, scale, ws)
+            return dq
+
+        return acc, dk, dv, finish
+
+    def _backward_no_keys(self, q, o, lse, do, dq, dk, dv, scale):
+        """A rank whose key range is empty adds nothing to dQ, but still takes part in the
+        all-reduce and, for bf16, converts the summed accumulator itself."""
+        m = self.m
+        if q.dtype == torch.float32:
+            return torch.zeros_like(q), dk, dv, lambda acc: acc
+        B, H, Nq, D = q.shape
+        # the phases take a key count >= 1: a one-key stand-in that PREPROCESS and FINALIZE never read
+        k1 = torch.zeros((B, H, 1, D), dtype=q.dtype, device=q.device)
+        g1 = torch.empty_like(k1)
+        ws = torch.empty(m.mea_attn_bwd_workspace_size(B, H, Nq, 1, D, q.dtype), dtype=torch.uint8, device=q.device)
+        m.mea_attn_bwd_phase(m.MEA_BWD_PREPROCESS, q, k1, k1, o, lse, do, dq, g1, g1, scale, ws)  # zeroes the acc
+        acc = ws[:B * H * Nq * D * 4].view(torch.float32)
+
+        def finish(summed):
+            m.mea_attn_bwd_phase(m.MEA_BWD_FINALIZE, q, k1, k1, o, lse, do, dq, g1, g1, scale, ws)
             return dq
 
         return acc, dk, dv, finish
@@ -76,7 +98,14 @@ def attention_forward_keysplit(q, k_local, v_local, scale=None, group=None, ops=
     """
     ops = CudaOps() if ops is None else ops
     scale = _scale(q, scale)
-    o_r, lse_r = ops.forward(q, k_local, v_local, scale)
+    if k_local.shape[2] == 0:
+        # a rank without keys (fewer keys than ranks) contributes the empty sum: weight
+        # e^{lse} = 0 in the merge, whatever its o; no kernel runs over zero keys
+        o_r = torch.zeros(q.shape[:3] + (v_local.shape[3],), dtype=q.dtype, device=q.device)
+        lse_dtype = torch.float64 if q.dtype == torch.float64 else torch.float32
+        lse_r = torch.full(q.shape[:3], float("-inf"), dtype=lse_dtype, device=q.device)
+    else:
+        o_r, lse_r = ops.forward(q, k_local, v_local, scale)
     world = dist.get_world_size(group)
     o_all = [torch.empty_like(o_r) for _ in range(world)]
     lse_all = [torch.empty_like(lse_r) for _ in range(world)]

@@ -238,7 +238,8 @@ mea_status_t mea_attn_fwd_fp8(const void* q, const void* k, const void* v,
  * Part r is mea_attn_fwd's output (o_r, lse_r) over the r-th key range; the
  * merge gives exactly the attention over all keys:
  *     lse = ln sum_r exp(lse_r),     o = sum_r exp(lse_r - lse) o_r.
- * A part with lse = -inf (no keys) contributes nothing.
+ * A part with lse = -inf (no keys) contributes nothing; a row whose parts all
+ * have lse = -inf has no keys at all and gets o = 0 and lse = -inf.
  *
  * o_parts, lse_parts: HOST arrays of R device pointers (1 <= R <= 16); each
  * o part is [B, H, Nq, D] in `dtype`, each lse part [B, H, Nq] fp32.  The
@@ -319,7 +320,10 @@ mea_status_t mea_attn_decode(const void* q, const void* k, const void* v,
  * MEA_NOALLOC_SCRATCH_BYTES are rejected with MEA_ERR_WORKSPACE and a message
  * in mea_last_error_message().  The first call on each device resolves the
  * array's device address (cudaGetSymbolAddress) with that device current; make
- * that first call before any stream capture.  All calls on a device share the
+ * that first call before any stream capture.  The address is remembered with
+ * the unique id of the CUDA context it belongs to: after cudaDeviceReset, or
+ * when another context becomes current, the next call resolves it again (so
+ * that call, too, belongs before any capture).  All calls on a device share the
  * one array: calls that overlap on the GPU (different streams, or different
  * host threads without ordering) race on it and give wrong gradients; calls
  * ordered on one stream are safe.  Each call clears the part that must start

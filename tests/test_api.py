@@ -141,6 +141,38 @@ def test_python_binding_rejects_bad_tensors(lib):
         m.mea_attn_fwd(q[0], q, q, q, torch.zeros(1, 1, 4), 0.125)
 
 
+@pytest.mark.parametrize("entry", ["mea_attn_bwd", "mea_attn_bwd_noalloc", "mea_attn_bwd_gqa"])
+def test_python_backward_rejects_mismatched_operands(lib, entry):
+    """The backward wrappers check k, v and lse against q before anything reaches the C side: the
+    kernels index every operand by q's sizes, so a smaller k or lse would be read past its end."""
+    import torch
+    import exact_memory_efficient_b200 as m
+    fn = getattr(m, entry)
+    q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 2, 8)
+
+    def call(k, lse_):
+        v, dk, dv = torch.zeros_like(k), torch.zeros_like(k), torch.zeros_like(k)
+        args = (q, k, v, q.clone(), lse_, q.clone(), q.clone(), dk, dv, 0.125)
+        return fn(*args) if entry == "mea_attn_bwd_noalloc" else fn(*args, None)
+
+    match = "k (must be|shape|dtype)" if entry != "mea_attn_bwd_gqa" else "k must be"
+    with pytest.raises(m.MeaError, match=match):
+        call(torch.zeros(1, 2, 8, 32, dtype=torch.bfloat16), lse)         # k's D differs from q's
+    with pytest.raises(m.MeaError, match=match):
+        call(torch.zeros(2, 2, 8, 64, dtype=torch.bfloat16), lse)         # k's B differs from q's
+    if entry != "mea_attn_bwd_gqa":                                        # (fewer k heads is GQA there)
+        with pytest.raises(m.MeaError, match=match):
+            call(torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16), lse)     # k's H differs from q's
+    k = torch.zeros(1, 2, 16, 64, dtype=torch.bfloat16)
+    with pytest.raises(m.MeaError, match="lse must be"):
+        call(k, lse.to(torch.bfloat16))                                    # lse not fp32
+    with pytest.raises(m.MeaError, match="lse must be"):
+        call(k, torch.zeros(1, 2, 4))                                      # lse shorter than Nq
+    with pytest.raises(m.MeaError, match="must be a contiguous CUDA tensor"):
+        call(k, lse)                                                       # consistent, but CPU tensors
+
+
 def test_gqa_argument_validation(lib):
     def fwd_gqa(H=4, Hkv=2, Nq=16, q=A, B=1):
         return lib.mea_attn_fwd_gqa(q, A, A, A, A, B, H, Hkv, Nq, 16, 64, ctypes.c_float(0.125), BF16, None)
@@ -258,3 +290,13 @@ def test_more_heads_than_the_launch_grid_is_unsupported():
     assert e.value.status == 2
     torch.cuda.synchronize()
     assert m.mea_last_device_error() == 0
+
+
+def test_noalloc_scratch_size_matches_header():
+    """The binding's MEA_NOALLOC_SCRATCH_BYTES (reported by the bench as resident memory) is the
+    header's #define."""
+    import exact_memory_efficient_b200 as m
+    with open(os.path.join(ROOT, "include", "mea_attn.h")) as f:
+        text = f.read()
+    a, b, c = re.search(r"#define MEA_NOALLOC_SCRATCH_BYTES \((\d+)u \* (\d+)u \* (\d+)u\)", text).groups()
+    assert m.MEA_NOALLOC_SCRATCH_BYTES == int(a) * int(b) * int(c)

@@ -66,6 +66,80 @@ def test_combine_skips_parts_without_keys():
     assert torch.equal(o, a) and torch.allclose(lse, la)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_combine_row_without_any_keys(dtype):
+    """Rows whose parts are all empty (lse = -inf everywhere) have no keys: the empty sum gives
+    lse = ln 0 = -inf and o = 0; the other rows merge as usual."""
+    import exact_memory_efficient_b200 as m
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    g = torch.Generator().manual_seed(5)
+    o_parts = [torch.randn(1, 2, 9, 64, generator=g).to(tdt) for _ in range(3)]
+    lse_parts = [torch.randn(1, 2, 9, generator=g) for _ in range(3)]
+    empty_rows = [0, 4, 8]
+    for lp in lse_parts:
+        lp[0, 1, empty_rows] = float("-inf")
+    o_parts[2][0, 1, empty_rows] = float("nan")    # an empty part's o is never read into the result
+    o = torch.empty(1, 2, 9, 64, dtype=tdt, device="cuda")
+    lse = torch.empty(1, 2, 9, device="cuda")
+    m.mea_attn_combine([x.cuda() for x in o_parts], [x.cuda() for x in lse_parts], o, lse)
+    assert m.mea_last_device_error() == m.MEA_OK
+    o, lse = to_np(o), to_np(lse)
+    assert np.all(o[0, 1, empty_rows] == 0.0) and np.all(np.isneginf(lse[0, 1, empty_rows]))
+    keep = [i for i in range(9) if i not in empty_rows]
+    with np.errstate(invalid="ignore"):   # the oracle's merge leaves the keyless rows undefined (compared apart)
+        ro, rl = oracle.combine_partials(np.stack([to_f64(x) for x in o_parts]),
+                                         np.stack([to_f64(x) for x in lse_parts]))
+    tol = BF16_O if dtype == "bf16" else (F32_O_MAX_ABS, None)
+    assert_close(o[0, 0], ro[0, 0], *tol, what="rows with keys, head 0")
+    assert_close(o[0, 1, keep], ro[0, 1, keep], *tol, what="rows with keys, head 1")
+    assert float(np.abs(lse[0, 1, keep] - rl[0, 1, keep]).max()) <= 1e-5 * max(1.0, float(np.abs(rl).max()))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_keysplit_rank_without_keys(dtype):
+    """Fewer keys than ranks: an emulated rank whose key range is empty runs no kernel over zero
+    keys, contributes o = 0, lse = -inf to the merge and a zero dQ partial to the sum, and (bf16)
+    finalises the summed dQ accumulator itself."""
+    from exact_memory_efficient_b200.keysplit import CudaOps
+    import exact_memory_efficient_b200 as m
+    w = custom(1, 2, 7, 3, 64, dtype)            # few rows, so that the gradients stay of order one
+    q, k, v, do = make_inputs(w, 25)
+    qd, kd, vd, dod = (x.cuda() for x in (q, k, v, do))
+    ops = CudaOps()
+    rs = [(0, 0), (0, 1), (1, 3), (3, 3)]       # four ranks over three keys: two ranks hold none
+    o_parts, lse_parts = [], []
+    for a, b in rs:
+        if b == a:   # what attention_forward_keysplit contributes for an empty range
+            o_parts.append(torch.zeros_like(qd))
+            lse_parts.append(torch.full(qd.shape[:3], float("-inf"), device="cuda"))
+        else:
+            o_r, l_r = ops.forward(qd, kd[:, :, a:b].contiguous(), vd[:, :, a:b].contiguous(), w.scale)
+            o_parts.append(o_r)
+            lse_parts.append(l_r)
+    o, lse = ops.combine(o_parts, lse_parts)
+    parts = [ops.backward_partial(qd, kd[:, :, a:b].contiguous(), vd[:, :, a:b].contiguous(), o, lse, dod, w.scale)
+             for a, b in rs]
+    total = sum(p[0] for p in parts)             # the all-reduce
+    for p in parts:
+        p[0].copy_(total)
+    dqs = [p[3](p[0]) for p in parts]
+    assert m.mea_last_device_error() == m.MEA_OK
+    rq, rk, rv, ro, rl = oracle.attention_backward(to_f64(q), to_f64(k), to_f64(v), to_f64(do), w.scale)
+    if dtype == "bf16":
+        assert_close(to_np(o), ro, *BF16_O, what="O")
+        for r, dq in enumerate(dqs):         # every rank, the empty ones too, ends with the full dq
+            assert_close(to_np(dq), rq, *BF16_GRAD, what=f"dQ rank {r}")
+        assert_close(to_np(torch.cat([p[1] for p in parts], dim=2)), rk, *BF16_GRAD, what="dK")
+        assert_close(to_np(torch.cat([p[2] for p in parts], dim=2)), rv, *BF16_GRAD, what="dV")
+    else:
+        assert_close(to_np(o), ro, F32_O_MAX_ABS, what="fp32 O")
+        for r, dq in enumerate(dqs):
+            assert_close(to_np(dq), rq, F32_O_MAX_ABS, what=f"fp32 dQ rank {r}")
+        assert_close(to_np(torch.cat([p[1] for p in parts], dim=2)), rk, F32_O_MAX_ABS, what="fp32 dK")
+        assert_close(to_np(torch.cat([p[2] for p in parts], dim=2)), rv, F32_O_MAX_ABS, what="fp32 dV")
+    assert_lse_close(to_np(lse), rl, to_f64(q), to_f64(k), w.scale)
+
+
 @pytest.mark.parametrize("B,H,Nq,Nk,D,R", [
     (1, 2, 300, 1000, 128, 2),
     (2, 3, 129, 777, 64, 3),
@@ -121,9 +195,9 @@ def test_split_backward_bf16(B, H, Nq, Nk, D, R):
                          vd[:, :, rs[0][0]:rs[0][1]].contiguous(), o, lse, dod, dq, dks[0], dvs[0], w.scale, wss[0])
     assert m.mea_last_device_error() == m.MEA_OK
     rq, rk, rv, _, _ = oracle.attention_backward(to_f64(q), to_f64(k), to_f64(v), to_f64(do), w.scale)
-    assert_close(to_np(dq), rq, *BF16_GRAD, what="split dQ", bf16_output=True)
-    assert_close(to_np(torch.cat(dks, dim=2)), rk, *BF16_GRAD, what="split dK", bf16_output=True)
-    assert_close(to_np(torch.cat(dvs, dim=2)), rv, *BF16_GRAD, what="split dV", bf16_output=True)
+    assert_close(to_np(dq), rq, *BF16_GRAD, what="split dQ")
+    assert_close(to_np(torch.cat(dks, dim=2)), rk, *BF16_GRAD, what="split dK")
+    assert_close(to_np(torch.cat(dvs, dim=2)), rv, *BF16_GRAD, what="split dV")
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -152,7 +226,7 @@ def test_keysplit_module_one_rank_nccl(dtype):
     if dtype == "bf16":
         assert_close(to_np(o), ro, *BF16_O, what="keysplit O")
         for name, g_, r_ in (("dQ", dq, rq), ("dK", dk, rk), ("dV", dv, rv)):
-            assert_close(to_np(g_), r_, *BF16_GRAD, what=f"keysplit {name}", bf16_output=True)
+            assert_close(to_np(g_), r_, *BF16_GRAD, what=f"keysplit {name}")
     else:
         assert_close(to_np(o), ro, F32_O_MAX_ABS, what="keysplit fp32 O")
         for name, g_, r_ in (("dQ", dq, rq), ("dK", dk, rk), ("dV", dv, rv)):

@@ -67,7 +67,7 @@ def _worker(rank, world, port, inputs, out_dir):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,Nk", [(2, 37), (3, 50)])
+@pytest.mark.parametrize("world,Nk", [(2, 37), (3, 50), (3, 2), (4, 1)])  # the last two: ranks without keys
 def test_keysplit_exchange_reaches_full_attention(tmp_path, world, Nk):
     g = torch.Generator().manual_seed(world)
     q = torch.randn(1, 2, 6, 8, generator=g, dtype=torch.float64)
@@ -90,6 +90,7 @@ def test_keysplit_exchange_reaches_full_attention(tmp_path, world, Nk):
         np.testing.assert_allclose(d["dk"].numpy(), rk[:, :, a:b], atol=1e-12)
         np.testing.assert_allclose(d["dv"].numpy(), rv[:, :, a:b], atol=1e-12)
     assert covered[0][0] == 0 and covered[-1][1] == Nk
+    assert (Nk >= world) == all(b > a for a, b in covered)
     assert all(covered[i][1] == covered[i + 1][0] for i in range(world - 1))
 
 
