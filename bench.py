@@ -203,6 +203,102 @@ def cpu_oracle_sample(w, seed=0, q_rows=4096, min_seconds=0.0):
                                           f"heads, {q_rows} of {w.Nq} query rows x all {w.Nk} keys each, D={w.D}")
 
 
+def time_back_to_back(call, sets, stream, reps=30):
+    """Device time of one call (microseconds): `reps` back-to-back calls over the input sets
+    in turn, queued behind a sleep kernel so that the host has enqueued them all before the
+    GPU reaches them, bracketed by one event pair on the launching stream."""
+    for st in sets:
+        call(st)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(40_000_000)
+    e0.record(stream)
+    for r in range(reps):
+        call(sets[r % len(sets)])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps * 1e3
+
+
+def naive_attention(q, k, v, scale):
+    """The materialised-scores attention the method avoids: S = scale Q K^T, P = softmax(S),
+    O = P V, as three plain PyTorch operations in the inputs' dtype (memory baseline only)."""
+    s = torch.matmul(q, k.transpose(-1, -2)) * scale
+    p = torch.softmax(s, dim=-1)
+    return torch.matmul(p, v)
+
+
+def measure_memory(m, w, dev, stream):
+    """Peak device memory beyond inputs and outputs, measured by the caching allocator's peak
+    (torch.cuda.max_memory_allocated) for four runs of the workload: the naive materialised
+    attention forward, the same with an autograd backward, this library's forward (its extra
+    is lse) and its forward + backward (lse + the backward workspace).  The library allocates
+    nothing itself, which the driver's free-memory count around its calls confirms."""
+    scale = w.scale
+    q_h, k_h, v_h, do_h = make_inputs(w, 0)
+    out = {}
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+    def peak_above(base):
+        torch.cuda.synchronize()
+        return torch.cuda.max_memory_allocated(dev) - base
+
+    # naive forward: the extra is everything beyond q, k, v and the output o
+    q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
+    torch.cuda.reset_peak_memory_stats(dev)
+    base = torch.cuda.memory_allocated(dev)
+    with torch.no_grad():
+        o = naive_attention(q, k, v, scale)
+    out["naive_fwd_peak_bytes"] = peak_above(base) - o.numel() * o.element_size()
+    del o
+    # naive forward + autograd backward: beyond q, k, v, dO, o and the three gradients
+    qg, kg, vg = (x.clone().requires_grad_(True) for x in (q, k, v))
+    do = do_h.to(dev)
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    torch.cuda.reset_peak_memory_stats(dev)
+    base = torch.cuda.memory_allocated(dev)
+    o = naive_attention(qg, kg, vg, scale)
+    o.backward(do)
+    grads = sum(x.grad.numel() * x.grad.element_size() for x in (qg, kg, vg))
+    out["naive_fwdbwd_peak_bytes"] = peak_above(base) - o.numel() * o.element_size() - grads
+    del o, qg, kg, vg
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    # this library: outputs allocated first, then the extra (lse, workspace) inside the window
+    o = torch.empty_like(q)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info(dev)[0]
+    torch.cuda.reset_peak_memory_stats(dev)
+    base = torch.cuda.memory_allocated(dev)
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+    m.mea_attn_fwd(q, k, v, o, lse, scale, stream)
+    out["ours_fwd_peak_bytes"] = peak_above(base)
+    ws = torch.empty(m.mea_attn_bwd_workspace_size(w.B, w.H, w.Nq, w.Nk, w.D), dtype=torch.uint8, device=dev)
+    m.mea_attn_bwd(q, k, v, o, lse, do, dq, dk, dv, scale, ws, stream)
+    out["ours_fwdbwd_peak_bytes"] = peak_above(base)
+    torch.cuda.synchronize()
+    # device memory taken between the two snapshots by anything (the allocator's new
+    # segments for lse and the workspace, and any allocation inside the library)
+    out["ours_driver_free_delta_bytes"] = int(free0 - torch.cuda.mem_get_info(dev)[0])
+    out["ours_allocator_extra_bytes"] = int(lse.numel() * 4 + ws.numel())
+    out["naive_over_ours_fwd"] = round(out["naive_fwd_peak_bytes"] / out["ours_fwd_peak_bytes"], 1)
+    out["naive_over_ours_fwdbwd"] = round(out["naive_fwdbwd_peak_bytes"] / out["ours_fwdbwd_peak_bytes"], 1)
+    out["pages_tpu_ratios"] = {"inference": 59, "differentiation": 32, "n": 16384, "hardware": "TPUv3"}
+    out["static_noalloc_scratch_bytes"] = int(m.MEA_NOALLOC_SCRATCH_BYTES)
+    out["note"] = ("peaks from torch.cuda.max_memory_allocated above inputs and outputs; naive = bf16 "
+                   "matmul -> softmax -> matmul (autograd for the backward); the static scratch of "
+                   "mea_attn_bwd_noalloc is resident on every device that loads the library, whether "
+                   "or not that entry point is called, and is listed apart")
+    del q, k, v, do, o, dq, dk, dv, lse, ws
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -456,21 +552,8 @@ def run_ours(args):
             ws_n = m.mea_attn_decode_workspace_size(wd.B, wd.H, wd.H_kv, wd.Nq, wd.Nk, wd.D, wd.torch_dtype)
             wsd = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=dev)
 
-            def time_calls(call, reps=30):
-                for st in sets:
-                    call(*st)
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                torch.cuda.synchronize()
-                torch.cuda._sleep(40_000_000)
-                e0.record(stream)
-                for r in range(reps):
-                    call(*sets[r % 3])
-                e1.record(stream)
-                torch.cuda.synchronize()
-                return e0.elapsed_time(e1) / reps * 1e3
-
-            us = time_calls(lambda q_, k_, v_, o_, l_: m.mea_attn_decode(q_, k_, v_, o_, l_, wd.scale, wsd))
-            us_fwd = time_calls(lambda q_, k_, v_, o_, l_: m.mea_attn_fwd_gqa(q_, k_, v_, o_, l_, wd.scale))
+            us = time_back_to_back(lambda s_: m.mea_attn_decode(*s_, wd.scale, wsd, stream), sets, stream)
+            us_fwd = time_back_to_back(lambda s_: m.mea_attn_fwd_gqa(*s_, wd.scale, stream), sets, stream)
             byts = sum(x.numel() * x.element_size() for x in sets[0])
             rows[f"{wname}_fwd"] = {"us": round(us, 2), "GB/s": round(byts / (us * 1e-6) / 1e9, 1),
                                     "frac_of_hbm": round(byts / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 3),
@@ -507,34 +590,40 @@ def run_ours(args):
                                   "note": f"mean of {reps}; inputs ({wg.H}+2x{wg.H_kv} heads) fit in L2"}
         del qg, kg, vg, dog, og, lg, wsg, grads
         # the head-dim-64 configurations (B4 H8 N4096 and B32 H8 N512), forward and
-        # backward through the public API; their inputs fit in L2
+        # backward through the public API, timed on the device like the decode rows:
+        # three copies of the inputs (3 x 67 MB > L2) used in turn, 30 back-to-back
+        # calls queued behind a sleep kernel and bracketed by one event pair.  Their
+        # roofline is max(compute at the measured bf16 peak, compulsory bytes at the
+        # measured HBM copy rate): the encoder-shaped batch sits near the ridge.
         for wname in ("mha_4k_bf16", "encoder_512_bf16"):
             wx = make_workload(wname)
-            qx, kx, vx, dox = (x.to(dev) for x in make_inputs(wx, 0))
-            ox, lx = m.attention_forward(qx, kx, vx, wx.scale)
+            sets = []
+            for copy in range(3):
+                qx, kx, vx, dox = (x.to(dev) for x in make_inputs(wx, copy))
+                ox, lx = m.attention_forward(qx, kx, vx, wx.scale)
+                sets.append((qx, kx, vx, dox, ox, lx, [torch.empty_like(x) for x in (qx, kx, vx)]))
             wsx = torch.empty(m.mea_attn_bwd_workspace_size(wx.B, wx.H, wx.Nq, wx.Nk, wx.D), dtype=torch.uint8,
                               device=dev)
-            gx = [torch.empty_like(x) for x in (qx, kx, vx)]
-            for _ in range(3):
-                m.mea_attn_fwd(qx, kx, vx, ox, lx, wx.scale)
-                m.mea_attn_bwd(qx, kx, vx, ox, lx, dox, *gx, wx.scale, wsx)
-            reps = 10
-            ev_x = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
-            for e in ev_x:
-                e[0].record(stream)
-                m.mea_attn_fwd(qx, kx, vx, ox, lx, wx.scale)
-                e[1].record(stream)
-                m.mea_attn_bwd(qx, kx, vx, ox, lx, dox, *gx, wx.scale, wsx)
-                e[2].record(stream)
-            torch.cuda.synchronize()
-            f_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev_x)
-            b_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev_x)
-            rows[f"{wname}_fwd"] = {"ms": round(f_ms, 4), "TFLOP/s": round(wx.fwd_flops() / (f_ms * 1e-3) / 1e12, 1),
-                                    "frac_of_peak": round(wx.fwd_flops() / (f_ms * 1e-3) / 1e12 / peak, 3)}
-            rows[f"{wname}_bwd"] = {"ms": round(b_ms, 4), "TFLOP/s": round(wx.bwd_flops() / (b_ms * 1e-3) / 1e12, 1),
-                                    "frac_of_peak": round(wx.bwd_flops() / (b_ms * 1e-3) / 1e12 / peak, 3),
-                                    "note": f"mean of {reps}; D={wx.D}, inputs fit in L2"}
-            del qx, kx, vx, dox, ox, lx, wsx, gx
+            f_us = time_back_to_back(lambda s_: m.mea_attn_fwd(s_[0], s_[1], s_[2], s_[4], s_[5], wx.scale, stream),
+                                     sets, stream)
+            b_us = time_back_to_back(lambda s_: m.mea_attn_bwd(s_[0], s_[1], s_[2], s_[4], s_[5], s_[3], *s_[6],
+                                                               wx.scale, wsx, stream), sets, stream)
+            elt = 2  # bf16
+            tensor_bytes = wx.B * wx.H * wx.Nq * wx.D * elt
+            rows_bytes = wx.B * wx.H * wx.Nq * 4
+            fwd_bytes = 4 * tensor_bytes + rows_bytes            # q, k, v read; o written; lse written
+            bwd_bytes = 8 * tensor_bytes + 2 * rows_bytes        # q, k, v, o, dO read; dq, dk, dv written; lse, D
+            for kind, us, flops, byts in (("fwd", f_us, wx.fwd_flops(), fwd_bytes),
+                                          ("bwd", b_us, wx.bwd_flops(), bwd_bytes)):
+                t_tensor = flops / (peak * 1e12) * 1e6
+                t_hbm = byts / (peaks["hbm_gbs"] * 1e9) * 1e6
+                rows[f"{wname}_{kind}"] = {
+                    "us": round(us, 2), "TFLOP/s": round(flops / (us * 1e-6) / 1e12, 1),
+                    "frac_of_peak": round(flops / (us * 1e-6) / 1e12 / peak, 3),
+                    "roofline_us": round(max(t_tensor, t_hbm), 2), "bound": "tensor" if t_tensor >= t_hbm else "hbm",
+                    "frac_of_roofline": round(max(t_tensor, t_hbm) / us, 3), "compulsory_bytes": byts,
+                    "note": f"D={wx.D}; 30 back-to-back calls over 3 input copies (> L2) behind a sleep kernel"}
+            del sets, wsx
         # merge of a 4-way key split of the step's workload (HBM-bound): reads four
         # [B,H,N,D] bf16 parts and their lse, writes the merged o and lse
         R = 4
@@ -583,11 +672,13 @@ def run_ours(args):
                                              "burst / 0.75 (S at 2x the bf16 rate, P V at bf16)"}
         del q8, k8, v8, o8, l8
 
-    # ---- extra memory versus a materialised-scores attention (arithmetic)
-    naive_scores = w.B * w.H * w.Nq * w.Nk * 4
+    # ---- extra memory versus a materialised-scores attention (measured peaks)
     memory = {"extra_bytes_ours": extra_bytes, "io_bytes": mem_io,
-              "naive_score_matrix_fp32_bytes": naive_scores,
-              "naive_over_ours": round(naive_scores / extra_bytes, 1)}
+              "naive_score_matrix_fp32_bytes": w.B * w.H * w.Nq * w.Nk * 4,
+              "static_noalloc_scratch_bytes": int(m.MEA_NOALLOC_SCRATCH_BYTES)}
+    if rank == 0 and not args.no_extras:
+        del q, k, v, do, o, dq, dk, dv, lse, ws
+        memory.update(measure_memory(m, w, dev, stream))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.no_extras:
