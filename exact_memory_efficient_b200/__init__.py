@@ -28,6 +28,7 @@ __all__ = [
     "MEA_ERR_CUDA", "MEA_ERR_TIMEOUT", "MEA_DTYPE_F32", "MEA_DTYPE_BF16",
     "MEA_BWD_ALL", "MEA_BWD_PREPROCESS", "MEA_BWD_MAIN", "MEA_BWD_FINALIZE", "MEA_NOALLOC_SCRATCH_BYTES",
     "mea_attn_fwd", "mea_attn_bwd", "mea_attn_bwd_phase", "mea_attn_bwd_workspace_size", "mea_attn_bwd_noalloc",
+    "mea_attn_bwd_accum", "mea_attn_bwd_accum_workspace_size", "mea_attn_accum_convert",
     "mea_attn_fwd_gqa", "mea_attn_bwd_gqa", "mea_attn_bwd_gqa_workspace_size", "mea_attn_fwd_fp8",
     "mea_attn_combine", "mea_attn_decode", "mea_attn_decode_workspace_size", "attention_decode",
     "mea_last_device_error",
@@ -91,6 +92,12 @@ def load_library() -> ctypes.CDLL:
     lib.mea_attn_bwd_phase.restype = i
     lib.mea_attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     lib.mea_attn_bwd_noalloc.restype = i
+    lib.mea_attn_bwd_accum_workspace_size.argtypes = [i, i, i, i, i, i, ctypes.POINTER(sz)]
+    lib.mea_attn_bwd_accum_workspace_size.restype = i
+    lib.mea_attn_bwd_accum.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
+    lib.mea_attn_bwd_accum.restype = i
+    lib.mea_attn_accum_convert.argtypes = [vp, vp, ctypes.c_longlong, f, i, vp]
+    lib.mea_attn_accum_convert.restype = i
     lib.mea_attn_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
     lib.mea_attn_fwd_gqa.restype = i
     lib.mea_attn_bwd_gqa_workspace_size.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(sz)]
@@ -245,6 +252,51 @@ def mea_attn_bwd_noalloc(q, k, v, o, lse, do, dq, dk, dv, scale: float, stream=N
                                               _ptr(dk), _ptr(dv), B, H, Nq, Nk, D, float(scale), _dtype_code(q),
                                               _stream_handle(stream))
     _check(st, "mea_attn_bwd_noalloc")
+
+
+def mea_attn_bwd_accum_workspace_size(B: int, H: int, Nq: int, Nk: int, D: int, dtype=torch.bfloat16) -> int:
+    out = ctypes.c_size_t(0)
+    code = MEA_DTYPE_BF16 if dtype == torch.bfloat16 else MEA_DTYPE_F32
+    st = load_library().mea_attn_bwd_accum_workspace_size(B, H, Nq, Nk, D, code, ctypes.byref(out))
+    _check(st, "mea_attn_bwd_accum_workspace_size")
+    return int(out.value)
+
+
+def mea_attn_bwd_accum(q, k, v, o, lse, do, dq_acc, dk_acc, dv_acc, scale: float, workspace, stream=None) -> None:
+    """C ``mea_attn_bwd_accum``: adds this key range's dS K, dS^T Q (both unscaled) and P^T dO to the
+    fp32 sums dq_acc [B,H,Nq,D], dk_acc, dv_acc [B,H,Nk,D]; o, lse are the merged results over all keys."""
+    B, H, Nq, D = _shape4(q, "q")
+    Bk, Hk, Nk, Dk = _shape4(k, "k")
+    if (Bk, Hk, Dk) != (B, H, D):
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_bwd_accum: k must be [B, H, Nk, D] with q's B, H and D")
+    for name, t, shape in (("v", v, k.shape), ("o", o, q.shape), ("do", do, q.shape)):
+        if tuple(t.shape) != tuple(shape) or t.dtype != q.dtype:
+            raise MeaError(MEA_ERR_INVALID_ARG, f"mea_attn_bwd_accum: {name} shape/dtype mismatch")
+    for name, t, shape in (("dq_acc", dq_acc, q.shape), ("dk_acc", dk_acc, k.shape), ("dv_acc", dv_acc, k.shape)):
+        if tuple(t.shape) != tuple(shape) or t.dtype != torch.float32:
+            raise MeaError(MEA_ERR_INVALID_ARG, f"mea_attn_bwd_accum: {name} must be fp32 shaped like q or k")
+    if lse is None or tuple(lse.shape) != (B, H, Nq) or lse.dtype != torch.float32:
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_bwd_accum: lse must be fp32 [B, H, Nq]")
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do), ("dq_acc", dq_acc), ("dk_acc", dk_acc),
+                    ("dv_acc", dv_acc), ("lse", lse)):
+        if not t.is_contiguous() or not t.is_cuda:
+            raise MeaError(MEA_ERR_INVALID_ARG, f"mea_attn_bwd_accum: {name} must be a contiguous CUDA tensor")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load_library().mea_attn_bwd_accum(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq_acc),
+                                            _ptr(dk_acc), _ptr(dv_acc), B, H, Nq, Nk, D, float(scale),
+                                            _dtype_code(q), _ptr(workspace), ws_bytes, _stream_handle(stream))
+    _check(st, "mea_attn_bwd_accum")
+
+
+def mea_attn_accum_convert(acc, out, mul: float, stream=None) -> None:
+    """C ``mea_attn_accum_convert``: out = mul * acc (fp32 sums to out's dtype, bf16 or fp32)."""
+    if acc.dtype != torch.float32 or acc.shape != out.shape or not acc.is_contiguous() or not out.is_contiguous():
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_accum_convert: acc fp32 and out of the same shape")
+    if not acc.is_cuda or not out.is_cuda:
+        raise MeaError(MEA_ERR_INVALID_ARG, "mea_attn_accum_convert: CUDA tensors")
+    st = load_library().mea_attn_accum_convert(_ptr(acc), _ptr(out), acc.numel(), float(mul), _dtype_code(out),
+                                                _stream_handle(stream))
+    _check(st, "mea_attn_accum_convert")
 
 
 def _gqa_shapes(q, k, where: str, check_device: bool = True):

@@ -454,6 +454,101 @@ mea_status_t mea_attn_bwd_phase(mea_bwd_phase_t phase, const void* q, const void
     return cuda_status(mea::launch_bwd_bf16(a, s, phases), "bwd_bf16 launch");
 }
 
+mea_status_t mea_attn_bwd_accum_workspace_size(int B, int H, int Nq, int Nk, int D, mea_dtype_t dtype,
+                                               size_t* bytes) {
+    if (bytes == nullptr) return MEA_ERR_INVALID_ARG;
+    mea_status_t st = common_checks(B, H, Nq, Nk, D, 1.0f, dtype);
+    if (st != MEA_OK) return st;
+    *bytes = round_up((size_t)B * H * Nq * sizeof(float), 256);   // the row term D_i
+    return MEA_OK;
+}
+
+mea_status_t mea_attn_bwd_accum(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                const void* dO, float* dq_acc, float* dk_acc, float* dv_acc, int B, int H, int Nq,
+                                int Nk, int D, float scale, mea_dtype_t dtype, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+    mea_status_t st = common_checks(B, H, Nq, Nk, D, scale, dtype);
+    if (st != MEA_OK) return st;
+    const int BH = B * H;
+    if (BH == 0 || Nq == 0 || Nk == 0) return MEA_OK;   // an empty query or key range adds nothing
+    if (!q || !k || !v || !o || !lse || !dO || !dq_acc || !dk_acc || !dv_acc) return MEA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) || !aligned16(dq_acc) ||
+        !aligned16(dk_acc) || !aligned16(dv_acc) || !aligned4(lse))
+        return MEA_ERR_MISALIGNED;
+    size_t need = 0;
+    if ((st = mea_attn_bwd_accum_workspace_size(B, H, Nq, Nk, D, dtype, &need)) != MEA_OK) return st;
+    if (workspace == nullptr || workspace_bytes < need) return MEA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MEA_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    if ((st = device_info(&dev)) != MEA_OK) return st;
+    if (BH > 65535) return MEA_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const unsigned phases = mea::kBwdPhasePre | mea::kBwdPhaseMain;
+    if (dtype == MEA_DTYPE_F32) {
+        mea::F32BwdArgs f;
+        f.q = static_cast<const float*>(q);
+        f.k = static_cast<const float*>(k);
+        f.v = static_cast<const float*>(v);
+        f.o = static_cast<const float*>(o);
+        f.dO = static_cast<const float*>(dO);
+        f.lse = lse;
+        f.dq = dq_acc;
+        f.dk = dk_acc;
+        f.dv = dv_acc;
+        f.delta = static_cast<float*>(workspace);
+        f.BH = BH;
+        f.Nq = Nq;
+        f.Nk = Nk;
+        f.D = D;
+        f.scale = scale;
+        f.accumulate = true;
+        auto rows_per_cta = [&](int rows) {
+            int r = 8;
+            while (r > 1 && (long long)BH * ((rows + r - 1) / r) < 2LL * dev->sm_count) r /= 2;
+            return r;
+        };
+        f.q_rows_per_cta = rows_per_cta(Nq);
+        f.k_rows_per_cta = rows_per_cta(Nk);
+        return cuda_status(mea::launch_bwd_f32(f, s, phases), "bwd_f32 accumulate launch");
+    }
+    mea::Bf16BwdArgs a;
+    if ((st = make_map(&a.tm_q, q, BH, Nq, D)) != MEA_OK) return st;
+    if ((st = make_map(&a.tm_k, k, BH, Nk, D)) != MEA_OK) return st;
+    if ((st = make_map(&a.tm_v, v, BH, Nk, D)) != MEA_OK) return st;
+    if ((st = make_map(&a.tm_do, dO, BH, Nq, D)) != MEA_OK) return st;
+    // dS K goes straight into the caller's fp32 sum by the TMA reduce-adds
+    if ((st = make_map_f32_acc(&a.tm_dq_acc, dq_acc, BH, Nq, D)) != MEA_OK) return st;
+    a.o = static_cast<const uint16_t*>(o);
+    a.dO = static_cast<const uint16_t*>(dO);
+    a.lse = lse;
+    a.dq = nullptr;
+    a.dk = nullptr;
+    a.dv = nullptr;
+    a.dq_acc = nullptr;   // the preprocess phase leaves the caller's sum alone
+    a.delta = static_cast<float*>(workspace);
+    a.dk_acc = dk_acc;
+    a.dv_acc = dv_acc;
+    a.BH = BH;
+    a.Nq = Nq;
+    a.Nk = Nk;
+    a.D = D;
+    a.scale = scale;
+    return cuda_status(mea::launch_bwd_bf16(a, s, phases), "bwd_bf16 accumulate launch");
+}
+
+mea_status_t mea_attn_accum_convert(const float* acc, void* out, long long n, float mul, mea_dtype_t dtype,
+                                    void* stream) {
+    if (n < 0 || !std::isfinite(mul)) return MEA_ERR_INVALID_ARG;
+    if (dtype != MEA_DTYPE_F32 && dtype != MEA_DTYPE_BF16) return MEA_ERR_UNSUPPORTED;
+    if (n == 0) return MEA_OK;
+    if (n % 4 != 0) return fail(MEA_ERR_UNSUPPORTED, "mea_attn_accum_convert", "n must be a multiple of 4");
+    if (!acc || !out) return MEA_ERR_INVALID_ARG;
+    if (!aligned16(acc) || !aligned16(out)) return MEA_ERR_MISALIGNED;
+    return cuda_status(mea::launch_accum_convert(acc, out, n, mul, dtype == MEA_DTYPE_BF16,
+                                                 static_cast<cudaStream_t>(stream)),
+                       "accum_convert launch");
+}
+
 mea_status_t mea_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                           const void* dO, void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int D,
                           float scale, mea_dtype_t dtype, void* workspace, size_t workspace_bytes, void* stream) {

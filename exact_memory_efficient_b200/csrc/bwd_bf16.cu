@@ -83,6 +83,7 @@ __global__ void bwd_pre_kernel(const uint16_t* __restrict__ o, const uint16_t* _
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (lane == 0) delta[row] = acc;
+    if (dq_acc == nullptr) return;   // accumulating callers own (and keep) their dQ accumulator
     float4* z = reinterpret_cast<float4*>(dq_acc + row * D);
     for (int c = lane; c < D / 4; c += 32) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
@@ -98,6 +99,22 @@ __global__ void bwd_dq_final_kernel(const float* __restrict__ dq_acc, uint16_t* 
     r.x = pack_bf16x2(a.x * scale, a.y * scale);
     r.y = pack_bf16x2(a.z * scale, a.w * scale);
     reinterpret_cast<uint2*>(dq)[i] = r;
+}
+
+// fp32 accumulator -> output dtype: out = mul * acc (bf16 round to nearest even, or fp32)
+__global__ void accum_convert_kernel(const float* __restrict__ acc, void* __restrict__ out, long long n4, float mul,
+                                     bool bf16) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n4) return;
+    const float4 a = reinterpret_cast<const float4*>(acc)[i];
+    if (bf16) {
+        uint2 r;
+        r.x = pack_bf16x2(a.x * mul, a.y * mul);
+        r.y = pack_bf16x2(a.z * mul, a.w * mul);
+        reinterpret_cast<uint2*>(out)[i] = r;
+    } else {
+        reinterpret_cast<float4*>(out)[i] = make_float4(a.x * mul, a.y * mul, a.z * mul, a.w * mul);
+    }
 }
 
 // ----------------------------------------------------------------- main
@@ -145,8 +162,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const __grid_constant__ CUtensorMap tm_dq, const float* __restrict__ lse,
-                const float* __restrict__ delta, uint16_t* __restrict__ dk, uint16_t* __restrict__ dv, int Nq,
-                int Nk, float scale) {
+                const float* __restrict__ delta, uint16_t* __restrict__ dk, uint16_t* __restrict__ dv,
+                float* __restrict__ dk_acc, float* __restrict__ dv_acc, int Nq, int Nk, float scale) {
     using Cfg = BwdCfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
     BwdBarriers* bars = reinterpret_cast<BwdBarriers*>(smem + Cfg::offBars);
@@ -405,21 +422,36 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!(ok = do_ds(i))) break;
             if (i + 1 < n_q && !(ok = do_p(i + 1))) break;
         }
-        // ---- epilogue: dV, dK (scaled) rows of this CTA's keys
+        // ---- epilogue: dV, dK (scaled) rows of this CTA's keys, or, for an
+        //      accumulating caller, dV and the unscaled dS^T Q added to its fp32 sums
         if (ok && mbar_wait(&bars->final_done, 0, abort_flag)) {
             tc_fence_after();
             const int key = n0 + kr;
+            const bool accumulate = dk_acc != nullptr;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 const unsigned col = (which == 0 ? Cfg::colDV : Cfg::colDK) + g * (D / 2);
-                const float mul = (which == 0) ? 1.f : scale;
-                uint16_t* dst = (which == 0 ? dv : dk) + ((size_t)bh * Nk + key) * D + g * (D / 2);
+                const float mul = (which == 0 || accumulate) ? 1.f : scale;
+                const size_t off = ((size_t)bh * Nk + key) * D + g * (D / 2);
+                uint16_t* dst = (which == 0 ? dv : dk) + off;
+                float* fdst = accumulate ? (which == 0 ? dv_acc : dk_acc) + off : nullptr;
 #pragma unroll
                 for (int c0 = 0; c0 < D / 2; c0 += 32) {
                     uint32_t r[32];
                     tmem_ld32(tmem + lane_off + col + c0, r);
                     tmem_wait_ld();
-                    if (key_ok) {
+                    if (key_ok && accumulate) {
+                        float4* f4 = reinterpret_cast<float4*>(fdst + c0);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            float4 x = f4[c];
+                            x.x += __uint_as_float(r[4 * c]);
+                            x.y += __uint_as_float(r[4 * c + 1]);
+                            x.z += __uint_as_float(r[4 * c + 2]);
+                            x.w += __uint_as_float(r[4 * c + 3]);
+                            f4[c] = x;
+                        }
+                    } else if (key_ok) {
                         uint32_t pk[16];
 #pragma unroll
                         for (int c = 0; c < 16; ++c)
@@ -507,11 +539,19 @@ cudaError_t launch_main(const Bf16BwdArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     dim3 grid((a.Nk + kTile - 1) / kTile, a.BH, 1);
     kern<<<grid, kThreads, Cfg::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.tm_dq_acc, a.lse, a.delta,
-                                                      a.dk, a.dv, a.Nq, a.Nk, a.scale);
+                                                      a.dk, a.dv, a.dk_acc, a.dv_acc, a.Nq, a.Nk, a.scale);
     return cudaGetLastError();
 }
 
 }  // namespace
+
+cudaError_t launch_accum_convert(const float* acc, void* out, long long n, float mul, bool bf16, cudaStream_t stream) {
+    const long long n4 = n / 4;
+    if (n4 == 0) return cudaSuccess;
+    const int tpb = 256;
+    accum_convert_kernel<<<(unsigned)((n4 + tpb - 1) / tpb), tpb, 0, stream>>>(acc, out, n4, mul, bf16);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_bwd_bf16(const Bf16BwdArgs& a, cudaStream_t stream, unsigned phases) {
     const long long rows = (long long)a.BH * a.Nq;

@@ -74,7 +74,8 @@ template <int DPL>
 __global__ void __launch_bounds__(256)
 bwd_f32_dq_kernel(const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
                   const float* __restrict__ dO, const float* __restrict__ lse, const float* __restrict__ delta,
-                  float* __restrict__ dq, int Nq, int Nk, float scale, int rows_per_cta, int warps_per_row) {
+                  float* __restrict__ dq, int Nq, int Nk, float scale, int rows_per_cta, int warps_per_row,
+                  bool accumulate) {
     constexpr int D = 32 * DPL;
     __shared__ float part[8][32 * DPL];
     const unsigned lane = lane_id();
@@ -137,10 +138,17 @@ bwd_f32_dq_kernel(const float* __restrict__ q, const float* __restrict__ k, cons
     }
     sum_slices<DPL>(part, acc, warp, warps_per_row, slice, lane);
     if (row_ok && slice == 0) {
+        float* dst = dq + ((size_t)bh * Nq + row) * D + DPL * lane;
         float out[DPL];
+        if (accumulate) {   // fp32 sum of an accumulating caller: add the unscaled dS K
+            load_dims<DPL>(dst, out);
 #pragma unroll
-        for (int i = 0; i < DPL; ++i) out[i] = scale * acc[i];
-        store_dims<DPL>(dq + ((size_t)bh * Nq + row) * D + DPL * lane, out);
+            for (int i = 0; i < DPL; ++i) out[i] += acc[i];
+        } else {
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) out[i] = scale * acc[i];
+        }
+        store_dims<DPL>(dst, out);
     }
 }
 
@@ -149,7 +157,7 @@ __global__ void __launch_bounds__(256)
 bwd_f32_dkdv_kernel(const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
                     const float* __restrict__ dO, const float* __restrict__ lse, const float* __restrict__ delta,
                     float* __restrict__ dk, float* __restrict__ dv, int Nq, int Nk, float scale, int rows_per_cta,
-                    int warps_per_row) {
+                    int warps_per_row, bool accumulate) {
     constexpr int D = 32 * DPL;
     __shared__ float part[8][32 * DPL];
     const unsigned lane = lane_id();
@@ -224,10 +232,23 @@ bwd_f32_dkdv_kernel(const float* __restrict__ q, const float* __restrict__ k, co
     if (key_ok && slice == 0) {
         const size_t kj = ((size_t)bh * Nk + key) * D + DPL * lane;
         float out[DPL];
+        if (accumulate) {   // fp32 sums of an accumulating caller: add the unscaled dS^T Q and P^T dO
+            float prev[DPL];
+            load_dims<DPL>(dk + kj, out);
+            load_dims<DPL>(dv + kj, prev);
 #pragma unroll
-        for (int i = 0; i < DPL; ++i) out[i] = scale * acc_k[i];
-        store_dims<DPL>(dk + kj, out);
-        store_dims<DPL>(dv + kj, acc_v);
+            for (int i = 0; i < DPL; ++i) {
+                out[i] += acc_k[i];
+                prev[i] += acc_v[i];
+            }
+            store_dims<DPL>(dk + kj, out);
+            store_dims<DPL>(dv + kj, prev);
+        } else {
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) out[i] = scale * acc_k[i];
+            store_dims<DPL>(dk + kj, out);
+            store_dims<DPL>(dv + kj, acc_v);
+        }
     }
 }
 
@@ -245,13 +266,15 @@ cudaError_t launch_dpl(const F32BwdArgs& a, cudaStream_t stream, unsigned phases
         {
             dim3 grid((a.Nq + a.q_rows_per_cta - 1) / a.q_rows_per_cta, a.BH);
             bwd_f32_dq_kernel<DPL><<<grid, 256, 0, stream>>>(a.q, a.k, a.v, a.dO, a.lse, a.delta, a.dq, a.Nq, a.Nk,
-                                                             a.scale, a.q_rows_per_cta, 8 / a.q_rows_per_cta);
+                                                             a.scale, a.q_rows_per_cta, 8 / a.q_rows_per_cta,
+                                                             a.accumulate);
             cudaError_t e = cudaGetLastError();
             if (e != cudaSuccess) return e;
         }
         dim3 grid((a.Nk + a.k_rows_per_cta - 1) / a.k_rows_per_cta, a.BH);
         bwd_f32_dkdv_kernel<DPL><<<grid, 256, 0, stream>>>(a.q, a.k, a.v, a.dO, a.lse, a.delta, a.dk, a.dv, a.Nq,
-                                                           a.Nk, a.scale, a.k_rows_per_cta, 8 / a.k_rows_per_cta);
+                                                           a.Nk, a.scale, a.k_rows_per_cta, 8 / a.k_rows_per_cta,
+                                                           a.accumulate);
         return cudaGetLastError();
     }
     return cudaSuccess;

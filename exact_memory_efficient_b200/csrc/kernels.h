@@ -55,6 +55,9 @@ struct F32BwdArgs {
     float scale;
     int q_rows_per_cta;  // dQ kernel: query rows per CTA of 8 warps (1, 2, 4 or 8)
     int k_rows_per_cta;  // dK/dV kernel: key rows per CTA of 8 warps (1, 2, 4 or 8)
+    // Accumulating callers: dq, dk, dv are fp32 sums that receive the unscaled
+    // dS K, dS^T Q and P^T dO of this call (instead of being overwritten).
+    bool accumulate = false;
 };
 cudaError_t launch_bwd_f32(const F32BwdArgs& a, cudaStream_t stream, unsigned phases);
 
@@ -120,8 +123,12 @@ struct Bf16BwdArgs {
     uint16_t* dq;
     uint16_t* dk;
     uint16_t* dv;
-    float* dq_acc;  // workspace [BH, Nq, D] fp32
+    float* dq_acc;  // workspace [BH, Nq, D] fp32 (zeroed by the preprocess phase); nullptr: not zeroed
     float* delta;   // workspace [BH, Nq] fp32: sum_d dO * O
+    // Accumulating callers: dV and the unscaled dS^T Q are added to these fp32
+    // [BH, Nk, D] sums instead of being written to dk, dv (nullptr otherwise).
+    float* dk_acc = nullptr;
+    float* dv_acc = nullptr;
     int BH, Nq, Nk, D;
     float scale;
 };
@@ -130,5 +137,7 @@ constexpr unsigned kBwdPhasePre = 1u;    // delta = rowsum(dO o O); dQ accumulat
 constexpr unsigned kBwdPhaseMain = 2u;   // dK, dV; dQ accumulated in fp32
 constexpr unsigned kBwdPhaseFinal = 4u;  // dq = bf16(scale * dQ accumulator)
 cudaError_t launch_bwd_bf16(const Bf16BwdArgs& a, cudaStream_t stream, unsigned phases);
+// out[i] = mul * acc[i] as bf16 (round to nearest even) or fp32; n a multiple of 4.
+cudaError_t launch_accum_convert(const float* acc, void* out, long long n, float mul, bool bf16, cudaStream_t stream);
 
 }  // namespace mea

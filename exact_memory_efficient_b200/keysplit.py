@@ -87,6 +87,22 @@ class CudaOps:
         return acc, dk, dv, finish
 
 
+    # ---- accumulating backward (ring attention): fp32 sums that travel between calls
+    def accum_workspace(self, q, k):
+        B, H, Nq, D = q.shape
+        n = self.m.mea_attn_bwd_accum_workspace_size(B, H, Nq, k.shape[2], D, q.dtype)
+        return torch.empty(n, dtype=torch.uint8, device=q.device)
+
+    def backward_accumulate(self, q, k, v, o, lse, do, scale, dq_acc, dk_acc, dv_acc, workspace):
+        """dq_acc += dS K, dk_acc += dS^T Q, dv_acc += P^T dO over this key range (fp32, unscaled)."""
+        self.m.mea_attn_bwd_accum(q, k, v, o, lse, do, dq_acc, dk_acc, dv_acc, scale, workspace)
+
+    def accum_convert(self, acc, mul, dtype):
+        out = torch.empty(acc.shape, dtype=dtype, device=acc.device)
+        self.m.mea_attn_accum_convert(acc, out, mul)
+        return out
+
+
 def _scale(q, scale):
     return 1.0 / math.sqrt(q.shape[-1]) if scale is None else float(scale)
 

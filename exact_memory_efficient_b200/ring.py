@@ -16,12 +16,13 @@ may differ between ranks.  At step s it holds the key/value block of rank
 forward:   per step, the block's (o_b, lse_b) from the forward kernel is merged
            into the running (o, lse); the next block is received from rank
            r - 1 and the current one sent to rank r + 1 while it is computed.
-backward:  the key/value blocks travel again, each with fp32 accumulators of
-           its dk, dv.  Per step this rank adds the contributions of its
-           queries (P recomputed from the merged lse, so every contribution is
-           final) and passes block and accumulators on; a final send returns
-           every block's accumulators to its owner.  dq sums the per-step fp32
-           dQ accumulators locally.
+backward:  the key/value blocks travel again, each with fp32 sums of its dk,
+           dv.  Per step the library adds this rank's contributions
+           (mea_attn_bwd_accum: P recomputed from the merged lse, so every
+           contribution is final) to those sums and to the local fp32 dq sum,
+           and block and sums pass on; a final send returns every block's sums
+           to its owner, and mea_attn_accum_convert turns the three sums into
+           gradients.  No step does tensor arithmetic outside the library.
 
 The compute steps come from an ``ops`` object (the CUDA library by default) so
 that the exchange can run without a GPU; point-to-point transfers use
@@ -101,7 +102,9 @@ def ring_attention_backward(q, k_local, v_local, o, lse, do, scale=None, group=N
     """Gradients for this rank's shards: (dq, dk_local, dv_local).
 
     ``o`` and ``lse`` are this rank's results of ring_attention_forward.  Key and
-    value heads equal the query heads.
+    value heads equal the query heads.  The library adds every block's
+    contributions to fp32 sums (dq's stays here, dk's and dv's travel with their
+    block) and converts them to gradients once, at the end.
     """
     ops = CudaOps() if ops is None else ops
     scale = _scale(q, scale)
@@ -109,10 +112,10 @@ def ring_attention_backward(q, k_local, v_local, o, lse, do, scale=None, group=N
     lengths = _shard_lengths(k_local.shape[2], k_local.device, group)
     k_cur, v_cur = k_local.contiguous(), v_local.contiguous()
     acc_dtype = torch.float64 if q.dtype == torch.float64 else torch.float32
+    dq_acc = torch.zeros(q.shape, dtype=acc_dtype, device=q.device)
     dk_cur = torch.zeros(k_cur.shape, dtype=acc_dtype, device=k_cur.device)
     dv_cur = torch.zeros(v_cur.shape, dtype=acc_dtype, device=v_cur.device)
-    dq_acc = None
-    finish = None
+    workspace = ops.accum_workspace(q, k_cur)
     for s in range(world):
         n_next = lengths[(rank - s - 1) % world]
         shape = (k_cur.shape[0], k_cur.shape[1], n_next, k_cur.shape[3])
@@ -120,16 +123,10 @@ def ring_attention_backward(q, k_local, v_local, o, lse, do, scale=None, group=N
         if s + 1 < world:   # the next block travels while this one is computed
             (k_nxt, v_nxt), works = _exchange([k_cur, v_cur], [shape, shape], nxt, prv, group)
         if k_cur.shape[2] > 0:
-            acc_b, dk_b, dv_b, fin = ops.backward_partial(q, k_cur, v_cur, o, lse, do, scale)
-            dk_cur += dk_b.to(acc_dtype)
-            dv_cur += dv_b.to(acc_dtype)
-            if dq_acc is None:
-                dq_acc, finish = acc_b, fin
-            else:
-                dq_acc += acc_b
+            ops.backward_accumulate(q, k_cur, v_cur, o, lse, do, scale, dq_acc, dk_cur, dv_cur, workspace)
         if world > 1:
-            # the accumulators follow their block; after the last step every
-            # block's accumulators are back with their owner
+            # the sums follow their block; after the last step every block's
+            # sums are back with their owner
             (dk_nxt, dv_nxt), works_acc = _exchange([dk_cur, dv_cur], [shape, shape], nxt, prv, group)
             works += works_acc
         for w in works:
@@ -138,5 +135,5 @@ def ring_attention_backward(q, k_local, v_local, o, lse, do, scale=None, group=N
             dk_cur, dv_cur = dk_nxt, dv_nxt
         if s + 1 < world:
             k_cur, v_cur = k_nxt, v_nxt
-    dq = finish(dq_acc) if dq_acc is not None else torch.zeros_like(q)
-    return dq, dk_cur.to(k_local.dtype), dv_cur.to(v_local.dtype)
+    return (ops.accum_convert(dq_acc, scale, q.dtype), ops.accum_convert(dk_cur, scale, k_local.dtype),
+            ops.accum_convert(dv_cur, 1.0, v_local.dtype))

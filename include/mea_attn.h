@@ -302,6 +302,54 @@ mea_status_t mea_attn_decode(const void* q, const void* k, const void* v,
                              void* stream);
 
 /*
+ * Accumulating backward of one key range, for callers that split the keys
+ * (and queries) over several calls -- sequence-parallel attention whose
+ * key/value blocks visit every rank, as in the Ring Attention paragraph of
+ * "当注意力成为瓶颈从on困境到线性复杂度的技术突围" (section 分布式：突破单卡限制).
+ *
+ * P = exp(scale q k^T - lse) is recomputed from the given lse, which must be
+ * the merged lse over ALL keys (the checkpointing of "Self-attention Does Not
+ * Need O(n^2) Memory", English summary, method bullet on differentiation), and
+ * o the merged output.  Then every contribution of this key range is final and
+ * contributions of disjoint key (or query) ranges simply add, so this call adds
+ * to caller-owned fp32 sums:
+ *     dq_acc [B, H, Nq, D] += dS K,   dk_acc [B, H, Nk, D] += dS^T Q,
+ *     dv_acc [B, H, Nk, D] += P^T dO,   dS = P o (dO V^T - rowsum(dO o o)),
+ * WITHOUT the softmax scale on dq_acc and dk_acc (dQ = scale dq_acc,
+ * dK = scale dk_acc: see mea_attn_accum_convert).  The caller zeroes the sums
+ * before the first call; they stay fp32 over any number of calls.
+ *
+ * q, o, dO [B, H, Nq, D] and k, v [B, H, Nk, D] in `dtype` (bf16: D in {64,
+ * 128}; fp32: D in {32, 64, 96, 128}), lse [B, H, Nq] fp32; all device memory,
+ * 16-byte aligned (lse 4-byte), caller-owned.  `workspace` (256-byte aligned,
+ * at least mea_attn_bwd_accum_workspace_size bytes) holds the row term.  An
+ * empty query or key range adds nothing (MEA_OK).  Asynchronous on `stream`;
+ * dq_acc is summed by fp32 reduce-adds in no fixed order (bf16), dk_acc and
+ * dv_acc in a fixed order.  Errors: MEA_ERR_INVALID_ARG, MEA_ERR_UNSUPPORTED,
+ * MEA_ERR_MISALIGNED, MEA_ERR_WORKSPACE, MEA_ERR_CUDA.
+ */
+mea_status_t mea_attn_bwd_accum_workspace_size(int B, int H, int Nq, int Nk, int D, mea_dtype_t dtype,
+                                               size_t* bytes);
+mea_status_t mea_attn_bwd_accum(const void* q, const void* k, const void* v,
+                                const void* o, const float* lse, const void* dO,
+                                float* dq_acc, float* dk_acc, float* dv_acc,
+                                int B, int H, int Nq, int Nk, int D, float scale,
+                                mea_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/*
+ * out[i] = mul * acc[i] for i < n, written as `dtype` (bf16 rounded to nearest
+ * even, or fp32): turns the fp32 sums of mea_attn_bwd_accum into gradients
+ * (mul = scale for dq and dk, 1 for dv).  acc, out: device memory, 16-byte
+ * aligned; n a multiple of 4 (MEA_ERR_UNSUPPORTED otherwise).  Asynchronous on
+ * `stream`.  Errors: MEA_ERR_INVALID_ARG, MEA_ERR_UNSUPPORTED,
+ * MEA_ERR_MISALIGNED, MEA_ERR_CUDA.
+ */
+mea_status_t mea_attn_accum_convert(const float* acc, void* out, long long n, float mul, mea_dtype_t dtype,
+                                    void* stream);
+
+/*
+ * Backward pass that allocates nothing and takes no workspace./*
  * Backward pass that allocates nothing and takes no workspace.  The paper has
  * no counterpart: this is a deployment convenience of this library.
  *

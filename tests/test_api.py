@@ -300,3 +300,35 @@ def test_noalloc_scratch_size_matches_header():
         text = f.read()
     a, b, c = re.search(r"#define MEA_NOALLOC_SCRATCH_BYTES \((\d+)u \* (\d+)u \* (\d+)u\)", text).groups()
     assert m.MEA_NOALLOC_SCRATCH_BYTES == int(a) * int(b) * int(c)
+
+
+def test_accumulating_backward_argument_validation(lib):
+    """mea_attn_bwd_accum and mea_attn_accum_convert reject bad arguments before any launch."""
+    out = ctypes.c_size_t(0)
+    assert lib.mea_attn_bwd_accum_workspace_size(2, 3, 100, 50, 64, BF16, ctypes.byref(out)) == 0
+    assert out.value == 2 * 3 * 100 * 4 + (256 - (2 * 3 * 100 * 4) % 256) % 256   # the row term, 256-aligned
+    assert lib.mea_attn_bwd_accum_workspace_size(1, 1, 16, 16, 96, BF16, ctypes.byref(out)) == 2
+
+    def accum(ptrs=None, Nq=16, Nk=16, D=64, ws=A, ws_bytes=1 << 20, dtype=BF16):
+        p = ptrs if ptrs is not None else [A] * 9
+        return lib.mea_attn_bwd_accum(*p, 1, 2, Nq, Nk, D, ctypes.c_float(0.125), dtype, ws, ws_bytes, None)
+
+    assert accum(Nq=0) == 0                      # an empty query range adds nothing
+    assert accum(Nk=0) == 0                      # an empty key range adds nothing
+    assert accum(D=96) == 2                      # bf16 takes D in {64, 128}
+    assert accum(ptrs=[A] * 6 + [None, A, A]) == 1
+    assert accum(ptrs=[A] * 7 + [A + 4, A]) == 3  # a misaligned fp32 sum
+    assert accum(ws=None) == 4
+    assert accum(ws_bytes=16) == 4
+    assert accum(ws=A + 16) == 3                 # workspace not 256-byte aligned
+
+    def conv(acc=A, o=A, n=1024, mul=1.0, dtype=BF16):
+        return lib.mea_attn_accum_convert(acc, o, ctypes.c_longlong(n), ctypes.c_float(mul), dtype, None)
+
+    assert conv(n=0) == 0
+    assert conv(n=6) == 2                        # not a multiple of 4
+    assert conv(n=-4) == 1
+    assert conv(acc=None) == 1
+    assert conv(o=A + 8) == 3
+    assert conv(mul=float("inf")) == 1
+    assert conv(dtype=7) == 2

@@ -194,6 +194,21 @@ def test_rising_scores_rescale_often():
     full_check(qt, kt, vt, 1.0, "rising scores")
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_rising_scores_many_items(D):
+    """The rising-score construction over 160 heads (320 query-tile pairs, so persistent CTAs walk
+    two or three items each): the reference maximum moves in most key tiles of every item, and
+    each item starts from a fresh maximum while the previous item's last tile is still in flight."""
+    B, H, Nq, Nk = 40, 4, 512, 1000
+    rng = np.random.default_rng(9)
+    q = np.ones((B, H, Nq, D)) * 0.25 + rng.normal(0, 0.01, (B, H, Nq, D))
+    ramp = np.linspace(-1.0, 1.0, Nk)[None, None, :, None] * rng.choice([-1.0, 1.0], (B, H, 1, 1))
+    k = ramp * (4.0 * 128 / D) + rng.normal(0, 0.01, (B, H, Nk, D))
+    v = rng.normal(0, 1, (B, H, Nk, D))
+    qt, kt, vt = (torch.tensor(x, dtype=torch.bfloat16) for x in (q, k, v))
+    full_check(qt, kt, vt, 1.0 if D == 128 else 0.5, f"rising scores, many items, D={D}")
+
+
 @pytest.mark.parametrize("B,H,Nq,Nk,D", [
     (1, 2, 300, 700, 128),    # ragged query tail: the last CTA holds one tile
     (1, 2, 512, 700, 128),    # full tile pairs

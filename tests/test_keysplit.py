@@ -200,6 +200,49 @@ def test_split_backward_bf16(B, H, Nq, Nk, D, R):
     assert_close(to_np(torch.cat(dvs, dim=2)), rv, *BF16_GRAD, what="split dV")
 
 
+@pytest.mark.parametrize("dtype,B,H,Nq,Nk,D,q_cuts,k_cuts", [
+    ("bf16", 1, 2, 300, 1000, 128, [0, 128, 300], [0, 333, 700, 1000]),
+    ("bf16", 2, 1, 257, 513, 64, [0, 257], [0, 1, 200, 513]),      # a one-key range
+    ("f32", 1, 2, 120, 400, 64, [0, 70, 120], [0, 150, 400]),
+])
+def test_accumulating_backward(dtype, B, H, Nq, Nk, D, q_cuts, k_cuts):
+    """mea_attn_bwd_accum over every (query range, key range) pair with the merged o, lse: the fp32
+    sums, converted by mea_attn_accum_convert, are the full gradients (contributions of disjoint
+    ranges add); the sums start at zero and stay fp32 across the calls."""
+    import exact_memory_efficient_b200 as m
+    w = custom(B, H, Nq, Nk, D, dtype)
+    q, k, v, do = make_inputs(w, 27)
+    qd, kd, vd, dod = (x.cuda() for x in (q, k, v, do))
+    o, lse = m.attention_forward(qd, kd, vd, w.scale)
+    dq_acc = torch.zeros(qd.shape, dtype=torch.float32, device="cuda")
+    dk_acc = torch.zeros(kd.shape, dtype=torch.float32, device="cuda")
+    dv_acc = torch.zeros(vd.shape, dtype=torch.float32, device="cuda")
+    for qa, qb in zip(q_cuts[:-1], q_cuts[1:]):
+        qs = slice(qa, qb)
+        q_r, o_r, l_r, do_r = (x[:, :, qs].contiguous() for x in (qd, o, lse, dod))
+        dq_r = torch.zeros(q_r.shape, dtype=torch.float32, device="cuda")
+        for ka, kb in zip(k_cuts[:-1], k_cuts[1:]):
+            ks = slice(ka, kb)
+            k_r, v_r = kd[:, :, ks].contiguous(), vd[:, :, ks].contiguous()
+            dk_r, dv_r = dk_acc[:, :, ks].contiguous(), dv_acc[:, :, ks].contiguous()
+            ws = torch.empty(m.mea_attn_bwd_accum_workspace_size(B, H, qb - qa, kb - ka, D, qd.dtype),
+                             dtype=torch.uint8, device="cuda")
+            m.mea_attn_bwd_accum(q_r, k_r, v_r, o_r, l_r, do_r, dq_r, dk_r, dv_r, w.scale, ws)
+            dk_acc[:, :, ks] = dk_r      # the sums of a key range travel on to the next query range
+            dv_acc[:, :, ks] = dv_r
+        dq_acc[:, :, qs] = dq_r
+    grads = []
+    for acc, mul, like in ((dq_acc, w.scale, qd), (dk_acc, w.scale, kd), (dv_acc, 1.0, vd)):
+        out = torch.empty_like(like)
+        m.mea_attn_accum_convert(acc, out, mul)
+        grads.append(out)
+    assert m.mea_last_device_error() == m.MEA_OK
+    rq, rk, rv, _, _ = oracle.attention_backward(to_f64(q), to_f64(k), to_f64(v), to_f64(do), w.scale)
+    tol = BF16_GRAD if dtype == "bf16" else (F32_O_MAX_ABS, 1e-5)
+    for name, g_, r_ in (("dQ", grads[0], rq), ("dK", grads[1], rk), ("dV", grads[2], rv)):
+        assert_close(to_np(g_), r_, *tol, what=f"accumulated {name}")
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_keysplit_module_one_rank_nccl(dtype):
     """The library's own key-split path (exact_memory_efficient_b200.keysplit with its CUDA ops)

@@ -41,6 +41,21 @@ class OracleOps:
         dv = np.einsum("bhij,bhid->bhjd", p, don)
         return torch.from_numpy(dq), torch.from_numpy(dk), torch.from_numpy(dv), lambda acc: acc
 
+    # accumulating interface (ring attention): unscaled sums, converted at the end
+    def accum_workspace(self, q, k):
+        return None
+
+    def backward_accumulate(self, q, k, v, o, lse, do, scale, dq_acc, dk_acc, dv_acc, workspace):
+        qn, kn, vn, on, ln, don = (x.numpy() for x in (q, k, v, o, lse, do))
+        p = np.exp(scale * np.einsum("bhid,bhjd->bhij", qn, kn) - ln[..., None])
+        ds = p * (np.einsum("bhid,bhjd->bhij", don, vn) - (don * on).sum(-1, keepdims=True))
+        dq_acc += torch.from_numpy(np.einsum("bhij,bhjd->bhid", ds, kn))
+        dk_acc += torch.from_numpy(np.einsum("bhij,bhid->bhjd", ds, qn))
+        dv_acc += torch.from_numpy(np.einsum("bhij,bhid->bhjd", p, don))
+
+    def accum_convert(self, acc, mul, dtype):
+        return (acc * mul).to(dtype)
+
 
 def _free_port():
     with socket.socket() as s:

@@ -2,8 +2,8 @@
 
 Two gloo ranks share the one GPU.  Each rank's compute steps are the
 library's own (exact_memory_efficient_b200.keysplit.CudaOps: the forward, the
-combine and the backward's PREPROCESS / MAIN / FINALIZE phases) on device
-copies of the tensors, while the ring transfers move host copies between the
+combine, the accumulating backward and the conversion of its fp32 sums) on
+device copies of the tensors, while the ring transfers move host copies between the
 ranks.  Every launch is an ordinary independent launch: no kernel waits on the
 other rank; the ranks meet only on the host, in the transfers.  The oracle
 computes full attention over the whole sequence.
@@ -49,6 +49,19 @@ class HostCudaOps:
             return fin(acc).cpu()
 
         return acc.cpu(), dk.cpu(), dv.cpu(), finish
+
+    def accum_workspace(self, q, k):
+        return self.ops.accum_workspace(q.cuda(), k.cuda())
+
+    def backward_accumulate(self, q, k, v, o, lse, do, scale, dq_acc, dk_acc, dv_acc, workspace):
+        accs = [a.cuda() for a in (dq_acc, dk_acc, dv_acc)]
+        self.ops.backward_accumulate(q.cuda(), k.cuda(), v.cuda(), o.cuda(), lse.cuda(), do.cuda(), scale, *accs,
+                                     workspace)
+        for host, dev in zip((dq_acc, dk_acc, dv_acc), accs):
+            host.copy_(dev.cpu())
+
+    def accum_convert(self, acc, mul, dtype):
+        return self.ops.accum_convert(acc.cuda(), mul, dtype).cpu()
 
 
 def _free_port():
