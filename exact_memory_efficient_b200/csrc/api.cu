@@ -451,6 +451,7 @@ mea_status_t mea_attn_bwd_phase(mea_bwd_phase_t phase, const void* q, const void
     a.Nk = Nk;
     a.D = D;
     a.scale = scale;
+    a.sm_count = dev->sm_count;
     return cuda_status(mea::launch_bwd_bf16(a, s, phases), "bwd_bf16 launch");
 }
 
@@ -533,6 +534,7 @@ mea_status_t mea_attn_bwd_accum(const void* q, const void* k, const void* v, con
     a.Nk = Nk;
     a.D = D;
     a.scale = scale;
+    a.sm_count = dev->sm_count;
     return cuda_status(mea::launch_bwd_bf16(a, s, phases), "bwd_bf16 accumulate launch");
 }
 

@@ -61,6 +61,9 @@ constexpr int kTile = 128;
 constexpr int kThreads = 512;
 constexpr int kComputeThreads = 256;
 constexpr int kDrainThreads = 128;
+// Persistent backward CTAs pay off while an item's query loop is short
+// (B32 H8 N512: 12 % faster); at 32 query tiles per item they measured 18 % slower.
+constexpr int kBwdPersistMaxQTiles = 8;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------ pre
@@ -119,15 +122,20 @@ __global__ void accum_convert_kernel(const float* __restrict__ acc, void* __rest
 
 // ----------------------------------------------------------------- main
 
-template <int D>
+template <int D, bool PERSIST>
 struct BwdCfg {
     static constexpr int kKVBytes = kTile * D * 2;      // one K (or V, Q, dO) tile
     static constexpr int kDSBytes = kTile * kTile * 2;  // dS^T tile, bf16
     static constexpr int kStageBytes = 4 * 64 * 32 * 4; // dQ staging: 4 warps x [64 queries x 32 floats]
     static constexpr int kBoxBytes = 128 * 128;
+    // K/V buffers: persistent CTAs load the next item's K and V into the
+    // other buffer while the current item finishes.  V must follow K in each
+    // buffer (read as K^T rows 64..127 at D = 64).
+    static constexpr int kKVBufs = PERSIST ? 2 : 1;
+    static constexpr int kKVBufBytes = 2 * kKVBytes;
     static constexpr int offK = 0;
-    static constexpr int offV = kKVBytes;               // must follow K (read as K^T rows 64..127 at D = 64)
-    static constexpr int offQ = 2 * kKVBytes;           // Q_i ring, 2 stages
+    static constexpr int offV = kKVBytes;
+    static constexpr int offQ = kKVBufs * kKVBufBytes;  // Q_i ring, 2 stages
     static constexpr int offDO = offQ + 2 * kKVBytes;   // dO_i, single buffer (dead after dV(i))
     static constexpr int offDS = offDO + kKVBytes;
     static constexpr int offStage = offDS + kDSBytes;
@@ -140,7 +148,8 @@ struct BwdCfg {
 };
 
 struct BwdBarriers {
-    uint64_t kv_full;
+    uint64_t kv_full[2];
+    uint64_t kv_empty[2];
     uint64_t q_full[2];
     uint64_t q_empty[2];
     uint64_t do_full, do_empty;
@@ -148,6 +157,7 @@ struct BwdBarriers {
     uint64_t p_ready, ds_ready, dq_free;
     uint64_t stats[2];
     uint64_t final_done;
+    uint64_t acc_free;
     uint64_t drain;
     unsigned tmem_base;
     int abort_flag;
@@ -157,14 +167,21 @@ struct BwdBarriers {
 // occupies columns [64 g, 64 g + 32) of its region.
 __device__ __forceinline__ unsigned packed_col(int kk) { return (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8; }
 
-template <int D>
+// Work items are (batch*head, 128-key tile) pairs.  Without PERSIST each CTA
+// owns one (grid = key tiles x heads, as before); with PERSIST a grid of at
+// most one CTA per SM walks items c, c + G, c + 2G, ...: the next item's K, V
+// load into the other buffer and its first S^T is issued while the current
+// item's last tile and epilogue are still in flight.  The query tiles of all
+// of a CTA's items form one sequence T = li * n_q + i; every per-tile barrier
+// takes its phase from T.
+template <int D, bool PERSIST>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const __grid_constant__ CUtensorMap tm_dq, const float* __restrict__ lse,
                 const float* __restrict__ delta, uint16_t* __restrict__ dk, uint16_t* __restrict__ dv,
-                float* __restrict__ dk_acc, float* __restrict__ dv_acc, int Nq, int Nk, float scale) {
-    using Cfg = BwdCfg<D>;
+                float* __restrict__ dk_acc, float* __restrict__ dv_acc, int BH, int Nq, int Nk, float scale) {
+    using Cfg = BwdCfg<D, PERSIST>;
     extern __shared__ __align__(1024) uint8_t smem[];
     BwdBarriers* bars = reinterpret_cast<BwdBarriers*>(smem + Cfg::offBars);
     float* s_lse2 = reinterpret_cast<float*>(smem + Cfg::offStats);          // [2][128]
@@ -172,17 +189,27 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     const unsigned warp = warp_id();
     const unsigned lane = lane_id();
-    const int bh = blockIdx.y;
-    const int n0 = blockIdx.x * kTile;      // first key of this CTA
     const int n_q = (Nq + kTile - 1) / kTile;
+    const int n_kt = (Nk + kTile - 1) / kTile;
+    const int n_items = PERSIST ? BH * n_kt : 1;
+    const int first = PERSIST ? (int)blockIdx.x : 0;
+    const int stride = PERSIST ? (int)gridDim.x : 1;
+    const int my_items = first < n_items ? (n_items - first + stride - 1) / stride : 0;
+    const int total = my_items * n_q;   // query tiles of this CTA over all its items
+    // (bh, first key) of this CTA's li-th item
+    auto item_bh = [&](int li) -> int { return PERSIST ? (first + li * stride) / n_kt : (int)blockIdx.y; };
+    auto item_n0 = [&](int li) -> int {
+        return (PERSIST ? (first + li * stride) % n_kt : (int)blockIdx.x) * kTile;
+    };
 
     if ((smem_u32(smem) & 1023u) != 0) {     // swizzle atoms need 1024-byte alignment
         if (threadIdx.x == 0) flag_timeout();
         return;
     }
     if (threadIdx.x == 0) {
-        mbar_init(&bars->kv_full, 1);
         for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars->kv_full[s], 1);
+            mbar_init(&bars->kv_empty[s], 1);
             mbar_init(&bars->q_full[s], 1);
             mbar_init(&bars->q_empty[s], 1);
         }
@@ -197,6 +224,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(&bars->stats[0], kDrainThreads);
         mbar_init(&bars->stats[1], kDrainThreads);
         mbar_init(&bars->final_done, 1);
+        mbar_init(&bars->acc_free, kComputeThreads);
         mbar_init(&bars->drain, 1);
         bars->abort_flag = 0;
         fence_mbar_init();
@@ -210,8 +238,6 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_after();
     const unsigned tmem = bars->tmem_base;
     volatile int* abort_flag = &bars->abort_flag;
-    uint8_t* sK = smem + Cfg::offK;
-    uint8_t* sV = smem + Cfg::offV;
     uint8_t* sQ = smem + Cfg::offQ;
     uint8_t* sDO = smem + Cfg::offDO;
     uint8_t* sDS = smem + Cfg::offDS;
@@ -224,47 +250,80 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
             prefetch_tmap(&tm_do);
-            mbar_arrive_expect_tx(&bars->kv_full, 2 * Cfg::kKVBytes);
-            for (int b = 0; b < D / 64; ++b) {
-                tma_load_3d(sK + b * Cfg::kBoxBytes, &tm_k, &bars->kv_full, b * 64, n0, bh);
-                tma_load_3d(sV + b * Cfg::kBoxBytes, &tm_v, &bars->kv_full, b * 64, n0, bh);
-            }
-            // Q_i: 2-stage ring (Q_{i+1} is read by S^T(i+1) before dK(i) frees Q_i).
-            // dO_i: single buffer, reloaded once dV(i) and dP^T(i) have read it.
-            auto load_q = [&](int i) {
-                mbar_arrive_expect_tx(&bars->q_full[i & 1], Cfg::kKVBytes);
-                for (int b = 0; b < D / 64; ++b)
-                    tma_load_3d(sQ + (i & 1) * Cfg::kKVBytes + b * Cfg::kBoxBytes, &tm_q, &bars->q_full[i & 1],
-                                b * 64, i * kTile, bh);
-            };
-            auto load_do = [&](int i) {
-                mbar_arrive_expect_tx(&bars->do_full, Cfg::kKVBytes);
-                for (int b = 0; b < D / 64; ++b)
-                    tma_load_3d(sDO + b * Cfg::kBoxBytes, &tm_do, &bars->do_full, b * 64, i * kTile, bh);
-            };
-            // dO_{i+1} is issued as soon as dV(i) has read dO_i, before Q_{i+2}
-            // (whose buffer frees only after dQ(i)).
-            int q_issued = 1, do_issued = 1;
-            load_q(0);
-            load_do(0);
-            if (n_q > 1) { load_q(1); q_issued = 2; }
-            for (int i = 0; i < n_q; ++i) {
-                if (i + 1 < n_q) {
-                    if (!mbar_wait(&bars->do_empty, i & 1, abort_flag)) break;
-                    load_do(i + 1);
-                    do_issued = i + 2;
+            // K, V of item li into buffer li % kKVBufs, once the item that used it last is done
+            auto load_kv = [&](int li) -> bool {
+                const int b = li % Cfg::kKVBufs;
+                if (li >= Cfg::kKVBufs &&
+                    !mbar_wait(&bars->kv_empty[b], ((li / Cfg::kKVBufs) - 1) & 1, abort_flag))
+                    return false;
+                uint8_t* sK = smem + b * Cfg::kKVBufBytes + Cfg::offK;
+                uint8_t* sV = smem + b * Cfg::kKVBufBytes + Cfg::offV;
+                const int bh = item_bh(li), n0 = item_n0(li);
+                mbar_arrive_expect_tx(&bars->kv_full[b], 2 * Cfg::kKVBytes);
+                for (int bx = 0; bx < D / 64; ++bx) {
+                    tma_load_3d(sK + bx * Cfg::kBoxBytes, &tm_k, &bars->kv_full[b], bx * 64, n0, bh);
+                    tma_load_3d(sV + bx * Cfg::kBoxBytes, &tm_v, &bars->kv_full[b], bx * 64, n0, bh);
                 }
-                if (i + 2 < n_q) {
-                    if (!mbar_wait(&bars->q_empty[i & 1], (i >> 1) & 1, abort_flag)) break;
-                    load_q(i + 2);
-                    q_issued = i + 3;
+                return true;
+            };
+            // Q_T: 2-stage ring (Q_{T+1} is read by S^T(T+1) before dK(T) frees Q_T).
+            // dO_T: single buffer, reloaded once dV(T) and dP^T(T) have read it.
+            // tile T's (query tile, batch*head) without a division per tile: the
+            // producer walks T in order, so the item is tracked incrementally
+            auto tile_of = [&](int T, int& i, int& bh) {
+                const int li = PERSIST ? T / n_q : 0;
+                i = T - li * n_q;
+                bh = item_bh(li);
+            };
+            auto load_q = [&](int T) {
+                int i, bh;
+                tile_of(T, i, bh);
+                mbar_arrive_expect_tx(&bars->q_full[T & 1], Cfg::kKVBytes);
+                for (int bx = 0; bx < D / 64; ++bx)
+                    tma_load_3d(sQ + (T & 1) * Cfg::kKVBytes + bx * Cfg::kBoxBytes, &tm_q, &bars->q_full[T & 1],
+                                bx * 64, i * kTile, bh);
+            };
+            auto load_do = [&](int T) {
+                int i, bh;
+                tile_of(T, i, bh);
+                mbar_arrive_expect_tx(&bars->do_full, Cfg::kKVBytes);
+                for (int bx = 0; bx < D / 64; ++bx)
+                    tma_load_3d(sDO + bx * Cfg::kBoxBytes, &tm_do, &bars->do_full, bx * 64, i * kTile, bh);
+            };
+            int q_issued = 0, do_issued = 0, kv_issued = 0;
+            bool ok = total > 0 && load_kv(0);
+            if (ok) {
+                kv_issued = 1;
+                load_q(0);
+                load_do(0);
+                q_issued = do_issued = 1;
+                if (total > 1) { load_q(1); q_issued = 2; }
+            }
+            for (int T = 0; ok && T < total; ++T) {
+                // the next item's K, V as soon as its buffer frees (persistent CTAs)
+                if (PERSIST && kv_issued < my_items && kv_issued * n_q <= T + n_q) {
+                    if (!(ok = load_kv(kv_issued))) break;
+                    ++kv_issued;
+                }
+                // dO_{T+1} as soon as dV(T) has read dO_T, before Q_{T+2}
+                // (whose buffer frees only after dK(T))
+                if (T + 1 < total) {
+                    if (!(ok = mbar_wait(&bars->do_empty, T & 1, abort_flag))) break;
+                    load_do(T + 1);
+                    do_issued = T + 2;
+                }
+                if (T + 2 < total) {
+                    if (!(ok = mbar_wait(&bars->q_empty[T & 1], (T >> 1) & 1, abort_flag))) break;
+                    load_q(T + 2);
+                    q_issued = T + 3;
                 }
             }
             // Never leave with copies in flight: wait until the last loads landed.
-            for (int i = (q_issued > 2 ? q_issued - 2 : 0); i < q_issued; ++i)
-                mbar_wait(&bars->q_full[i & 1], (i >> 1) & 1, nullptr);
+            for (int T = (q_issued > 2 ? q_issued - 2 : 0); T < q_issued; ++T)
+                mbar_wait(&bars->q_full[T & 1], (T >> 1) & 1, nullptr);
             if (do_issued > 0) mbar_wait(&bars->do_full, (do_issued - 1) & 1, nullptr);
-            mbar_wait(&bars->kv_full, 0, nullptr);
+            for (int li = (kv_issued > Cfg::kKVBufs ? kv_issued - Cfg::kKVBufs : 0); li < kv_issued; ++li)
+                mbar_wait(&bars->kv_full[li % Cfg::kKVBufs], (li / Cfg::kKVBufs) & 1, nullptr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
@@ -275,9 +334,10 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             constexpr unsigned idesc_g = make_idesc_bf16(128, D, 0, 1);     // dV, dK (A in TMEM)
             constexpr unsigned idesc_q = make_idesc_bf16(128, 128, 1, 1);   // dQ^T (A = K^T, B = dS^T, MN-major)
             constexpr unsigned idesc_k = make_idesc_bf16(128, D, 0, 1);     // dK (A = dS^T K-major, B = Q MN-major)
-            const uint32_t k_lo = desc_lo_kmajor(smem_u32(sK));             // K as A of S^T
-            const uint32_t kt_lo = desc_lo_mnmajor(smem_u32(sK));           // K^T as A of dQ^T
-            const uint32_t v_lo = desc_lo_kmajor(smem_u32(sV));
+            constexpr uint32_t kKVBufStep = Cfg::kKVBufBytes >> 4;          // start-field step between K/V buffers
+            const uint32_t k_lo0 = desc_lo_kmajor(smem_u32(smem + Cfg::offK));   // K as A of S^T
+            const uint32_t kt_lo0 = desc_lo_mnmajor(smem_u32(smem + Cfg::offK)); // K^T as A of dQ^T
+            const uint32_t v_lo0 = desc_lo_kmajor(smem_u32(smem + Cfg::offV));
             const uint32_t ds_lo = desc_lo_mnmajor(smem_u32(sDS));          // dS^T as B of dQ^T
             const uint32_t dsk_lo = desc_lo_kmajor(smem_u32(sDS));          // dS^T as A of dK
             const uint32_t do_k_lo = desc_lo_kmajor(smem_u32(sDO));         // dO as B of dP^T
@@ -287,61 +347,72 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             constexpr uint32_t kQStep = Cfg::kKVBytes >> 4;                  // start-field step between Q stages
             const unsigned tS = tmem + Cfg::colS, tDP = tmem + Cfg::colDP, tDV = tmem + Cfg::colDV,
                            tDK = tmem + Cfg::colDK, tDQ = tmem + Cfg::colDQ;
-            bool ok = mbar_wait(&bars->kv_full, 0, abort_flag);
-            // S^T(i) = K Q_i^T into the S columns (once Q_i has landed)
-            auto issue_s = [&](int i) -> bool {
-                if (!mbar_wait(&bars->q_full[i & 1], (i >> 1) & 1, abort_flag)) return false;
+            // S^T(T) = K Q_T^T into the S columns (once Q_T and the item's K have landed)
+            auto issue_s = [&](int T, int li, bool new_item) -> bool {
+                const int b = li % Cfg::kKVBufs;
+                if (new_item && !mbar_wait(&bars->kv_full[b], (li / Cfg::kKVBufs) & 1, abort_flag)) return false;
+                if (!mbar_wait(&bars->q_full[T & 1], (T >> 1) & 1, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t q_lo = q_k_lo0 + (uint32_t)(i & 1) * kQStep;
+                const uint32_t k_lo = k_lo0 + (uint32_t)b * kKVBufStep;
+                const uint32_t q_lo = q_k_lo0 + (uint32_t)(T & 1) * kQStep;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     mma_ss_lo(tS, k_lo + kmajor_step(kk), q_lo + kmajor_step(kk), idesc_t, kk > 0);
                 mma_commit(&bars->s_full);
                 return true;
             };
-            // Software pipeline: S^T(i+1) is issued right after dV(i) has been
-            // issued (which consumes P(i) from the same columns, in issue order),
-            // so the compute warps form P(i+1) while dK(i) and dQ(i) run.
-            if (ok) ok = issue_s(0);
-            for (int i = 0; ok && i < n_q; ++i) {
-                const uint32_t q_mn_lo = q_mn_lo0 + (uint32_t)(i & 1) * kQStep;
-                const unsigned acc0 = i > 0 ? 1u : 0u;
-                // dP^T = V dO_i^T  (D=128: dP columns held dQ_{i-1} until the dQ warps copied it out)
-                if (!(ok = mbar_wait(&bars->do_full, i & 1, abort_flag))) break;
-                if (Cfg::kDqInDp && i > 0) {
-                    if (!(ok = mbar_wait(&bars->dq_free, (i - 1) & 1, abort_flag))) break;
-                }
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_ss_lo(tDP, v_lo + kmajor_step(kk), do_k_lo + kmajor_step(kk), idesc_t, kk > 0);
-                mma_commit(&bars->dp_full);
-                // dV += P^T dO_i
-                if (!(ok = mbar_wait(&bars->p_ready, i & 1, abort_flag))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk)
-                    mma_ts_lo(tDV, tS + packed_col(kk), do_mn_lo + mnmajor_step(kk), idesc_g, (acc0 | kk) ? 1u : 0u);
-                mma_commit(&bars->do_empty);           // dO_i read by dP^T(i) and dV(i)
-                if (i + 1 < n_q && !(ok = issue_s(i + 1))) break;
-                // dQ_i^T = K^T dS^T first, so the dQ warps copy it out while dK
-                // runs; dK += dS^T Q_i then reads dS^T from shared memory too
-                if (!(ok = mbar_wait(&bars->ds_ready, i & 1, abort_flag))) break;
-                tc_fence_after();
-                if (!Cfg::kDqInDp && i > 0) {
-                    if (!(ok = mbar_wait(&bars->dq_free, (i - 1) & 1, abort_flag))) break;
+            bool ok = total > 0 && issue_s(0, 0, true);
+            for (int li = 0; ok && li < my_items; ++li) {
+                const uint32_t kvoff = (uint32_t)(li % Cfg::kKVBufs) * kKVBufStep;
+                const uint32_t kt_lo = kt_lo0 + kvoff;
+                const uint32_t v_lo = v_lo0 + kvoff;
+                for (int i = 0; i < n_q; ++i) {
+                    const int T = li * n_q + i;
+                    const uint32_t q_mn_lo = q_mn_lo0 + (uint32_t)(T & 1) * kQStep;
+                    const unsigned acc0 = i > 0 ? 1u : 0u;
+                    // dP^T = V dO_T^T  (D=128: dP columns held dQ_{T-1} until the dQ warps copied it out)
+                    if (!(ok = mbar_wait(&bars->do_full, T & 1, abort_flag))) break;
+                    if (Cfg::kDqInDp && T > 0) {
+                        if (!(ok = mbar_wait(&bars->dq_free, (T - 1) & 1, abort_flag))) break;
+                    }
                     tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ss_lo(tDP, v_lo + kmajor_step(kk), do_k_lo + kmajor_step(kk), idesc_t, kk > 0);
+                    mma_commit(&bars->dp_full);
+                    // dV += P^T dO_T; the item's first dV and dK overwrite the
+                    // accumulators, which the previous item's epilogue must have read
+                    if (!(ok = mbar_wait(&bars->p_ready, T & 1, abort_flag))) break;
+                    if (i == 0 && li > 0 && !(ok = mbar_wait(&bars->acc_free, (li - 1) & 1, abort_flag))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kTile / 16; ++kk)
+                        mma_ts_lo(tDV, tS + packed_col(kk), do_mn_lo + mnmajor_step(kk), idesc_g, (acc0 | kk) ? 1u : 0u);
+                    mma_commit(&bars->do_empty);           // dO_T read by dP^T(T) and dV(T)
+                    // Software pipeline: S^T(T+1) -- of this item, or of the next
+                    // one (persistent CTAs) -- right after dV(T)
+                    if (T + 1 < total && !(ok = issue_s(T + 1, (i + 1 < n_q) ? li : li + 1, i + 1 == n_q))) break;
+                    // dQ_T^T = K^T dS^T first, so the dQ warps copy it out while dK
+                    // runs; dK += dS^T Q_T then reads dS^T from shared memory too
+                    if (!(ok = mbar_wait(&bars->ds_ready, T & 1, abort_flag))) break;
+                    tc_fence_after();
+                    if (!Cfg::kDqInDp && T > 0) {
+                        if (!(ok = mbar_wait(&bars->dq_free, (T - 1) & 1, abort_flag))) break;
+                        tc_fence_after();
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < kTile / 16; ++kk)
+                        mma_ss_lo(tDQ, kt_lo + mnmajor_step(kk), ds_lo + mnmajor_step(kk), idesc_q, kk > 0);
+                    mma_commit(&bars->dq_full);
+#pragma unroll
+                    for (int kk = 0; kk < kTile / 16; ++kk)
+                        mma_ss_lo(tDK, dsk_lo + kmajor_step(kk), q_mn_lo + mnmajor_step(kk), idesc_k, (acc0 | kk) ? 1u : 0u);
+                    mma_commit(&bars->q_empty[T & 1]);
                 }
-#pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk)
-                    mma_ss_lo(tDQ, kt_lo + mnmajor_step(kk), ds_lo + mnmajor_step(kk), idesc_q, kk > 0);
-                mma_commit(&bars->dq_full);
-#pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk)
-                    mma_ss_lo(tDK, dsk_lo + kmajor_step(kk), q_mn_lo + mnmajor_step(kk), idesc_k, (acc0 | kk) ? 1u : 0u);
-                mma_commit(&bars->q_empty[i & 1]);
+                if (!ok) break;
+                mma_commit(&bars->final_done);                  // the item's dV, dK are complete
+                mma_commit(&bars->kv_empty[li % Cfg::kKVBufs]);  // and its K, V are no longer read
             }
-            if (ok) mma_commit(&bars->final_done);
             mma_commit(&bars->drain);
             mbar_wait(&bars->drain, 0, nullptr);
         }
@@ -352,13 +423,13 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int kr = sub * 32 + lane;                // key row within the tile (TMEM lane)
         const unsigned lane_off = (sub * 32u) << 16;
         const float c_log2 = scale * kLog2e;
-        const bool key_ok = (n0 + kr) < Nk;
         uint32_t pp[32];   // P^T of the current tile as packed bf16 pairs (exactly what dV used)
-        // ---- P^T = exp2(scale*log2e * S^T - lse2), query half g
-        auto do_p = [&](int t) -> bool {
-            const float* l2 = s_lse2 + (t & 1) * kTile + 64 * g;
-            if (!mbar_wait(&bars->stats[t & 1], (t >> 1) & 1, abort_flag)) return false;
-            if (!mbar_wait(&bars->s_full, t & 1, abort_flag)) return false;
+        // ---- P^T = exp2(scale*log2e * S^T - lse2), query half g, tile T of an item whose keys start at n0
+        auto do_p = [&](int T, int n0) -> bool {
+            const bool key_ok = (n0 + kr) < Nk;
+            const float* l2 = s_lse2 + (T & 1) * kTile + 64 * g;
+            if (!mbar_wait(&bars->stats[T & 1], (T >> 1) & 1, abort_flag)) return false;
+            if (!mbar_wait(&bars->s_full, T & 1, abort_flag)) return false;
             tc_fence_after();
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -380,11 +451,11 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_arrive(&bars->p_ready);
             return true;
         };
-        // ---- dS^T = P^T o (dP^T - delta): bf16 to TMEM (for dK) and to smem (for dQ)
-        auto do_ds = [&](int t) -> bool {
-            const float* dl = s_delta + (t & 1) * kTile + 64 * g;
-            if (!mbar_wait(&bars->dp_full, t & 1, abort_flag)) return false;
-            // dp_full(t) was committed after dQ(t-1) and dK(t-1), the readers of the dS buffer
+        // ---- dS^T = P^T o (dP^T - delta): bf16 to shared memory (for dQ and dK)
+        auto do_ds = [&](int T) -> bool {
+            const float* dl = s_delta + (T & 1) * kTile + 64 * g;
+            if (!mbar_wait(&bars->dp_full, T & 1, abort_flag)) return false;
+            // dp_full(T) was committed after dQ(T-1) and dK(T-1), the readers of the dS buffer
             tc_fence_after();
             // dS^T (keys x queries) in shared memory: MN-major operand, query block g,
             // row = key, 16-byte chunk c of the 128-byte row swizzled by (key mod 8).
@@ -415,33 +486,38 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_arrive(&bars->ds_ready);
             return true;
         };
-        // Order per tile: dS(t), then P(t+1) (overlapping dK(t), dQ(t) on the
-        // tensor cores); the dQ warps drain dQ(t) meanwhile.
-        bool ok = do_p(0);
-        for (int i = 0; ok && i < n_q; ++i) {
-            if (!(ok = do_ds(i))) break;
-            if (i + 1 < n_q && !(ok = do_p(i + 1))) break;
-        }
-        // ---- epilogue: dV, dK (scaled) rows of this CTA's keys, or, for an
-        //      accumulating caller, dV and the unscaled dS^T Q added to its fp32 sums
-        if (ok && mbar_wait(&bars->final_done, 0, abort_flag)) {
+        // Order per tile: dS(T), then P(T+1) (overlapping dK(T), dQ(T) on the
+        // tensor cores, and, at the end of an item, its epilogue); the dQ warps
+        // drain dQ(T) meanwhile.
+        bool ok = total > 0 && do_p(0, item_n0(0));
+        for (int li = 0; ok && li < my_items; ++li) {
+            const int n0 = item_n0(li);
+            for (int i = 0; i < n_q; ++i) {
+                const int T = li * n_q + i;
+                if (!(ok = do_ds(T))) break;
+                if (T + 1 < total && !(ok = do_p(T + 1, (i + 1 < n_q) ? n0 : item_n0(li + 1)))) break;
+            }
+            if (!ok) break;
+            // ---- epilogue of the item: dV, dK (scaled) rows of its keys, or, for an
+            //      accumulating caller, dV and the unscaled dS^T Q added to its fp32 sums
+            if (!(ok = mbar_wait(&bars->final_done, li & 1, abort_flag))) break;
             tc_fence_after();
+            const int bh = item_bh(li);
             const int key = n0 + kr;
+            const bool key_ok = key < Nk;
             const bool accumulate = dk_acc != nullptr;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 const unsigned col = (which == 0 ? Cfg::colDV : Cfg::colDK) + g * (D / 2);
                 const float mul = (which == 0 || accumulate) ? 1.f : scale;
                 const size_t off = ((size_t)bh * Nk + key) * D + g * (D / 2);
-                uint16_t* dst = (which == 0 ? dv : dk) + off;
-                float* fdst = accumulate ? (which == 0 ? dv_acc : dk_acc) + off : nullptr;
 #pragma unroll
                 for (int c0 = 0; c0 < D / 2; c0 += 32) {
                     uint32_t r[32];
                     tmem_ld32(tmem + lane_off + col + c0, r);
                     tmem_wait_ld();
                     if (key_ok && accumulate) {
-                        float4* f4 = reinterpret_cast<float4*>(fdst + c0);
+                        float4* f4 = reinterpret_cast<float4*>((which == 0 ? dv_acc : dk_acc) + off + c0);
 #pragma unroll
                         for (int c = 0; c < 8; ++c) {
                             float4 x = f4[c];
@@ -456,12 +532,15 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                         for (int c = 0; c < 16; ++c)
                             pk[c] = pack_bf16x2(__uint_as_float(r[2 * c]) * mul, __uint_as_float(r[2 * c + 1]) * mul);
-                        uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+                        uint4* d4 = reinterpret_cast<uint4*>((which == 0 ? dv : dk) + off + c0);
 #pragma unroll
                         for (int c = 0; c < 4; ++c) d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
                     }
                 }
             }
+            // dV, dK have been read: the next item's first dV and dK may overwrite them
+            tc_fence_before();
+            mbar_arrive(&bars->acc_free);
         }
     } else if (warp >= 12) {
         // ------------------------------------------------ dQ warps (+ lse/D staging)
@@ -470,18 +549,17 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const unsigned lane_off = (sub * 32u) << 16;
         const bool active = d < D;                     // D = 64: lanes 64..127 hold nothing useful
         const int j = threadIdx.x - 384;               // 0..127
-        const float* lse_h = lse + (size_t)bh * Nq;
-        const float* delta_h = delta + (size_t)bh * Nq;
         float* stage = reinterpret_cast<float*>(sStage + sub * 8192);   // this warp: 64 rows x 32 floats
-        auto stage_stats = [&](int t) {
-            const int row = t * kTile + j;
-            s_lse2[(t & 1) * kTile + j] = (row < Nq) ? lse_h[row] * kLog2e : INFINITY;
-            s_delta[(t & 1) * kTile + j] = (row < Nq) ? delta_h[row] : 0.f;
-            mbar_arrive(&bars->stats[t & 1]);
+        auto stage_stats = [&](int T, int li, int i) {
+            const size_t base = (size_t)item_bh(li) * Nq;
+            const int row = i * kTile + j;
+            s_lse2[(T & 1) * kTile + j] = (row < Nq) ? lse[base + row] * kLog2e : INFINITY;
+            s_delta[(T & 1) * kTile + j] = (row < Nq) ? delta[base + row] : 0.f;
+            mbar_arrive(&bars->stats[T & 1]);
         };
         // one half (64 queries) of dQ^T from registers to this warp's staging
         // buffer as [query][32 head dims], then one TMA reduce-add (not waited for)
-        auto stage_and_reduce = [&](const uint32_t (&v)[64], int q0) {
+        auto stage_and_reduce = [&](const uint32_t (&v)[64], int q0, int bh) {
             if (active) {
 #pragma unroll
                 for (int c = 0; c < 64; ++c) stage[c * 32 + lane] = __uint_as_float(v[c]);
@@ -497,26 +575,39 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (lane == 0) bulk_wait_read_all();
             __syncwarp();
         };
-        stage_stats(0);
-        if (n_q > 1) stage_stats(1);
+        // (item, query tile) of tile T + 2, advanced incrementally
+        int s_li = 0, s_i = 0;
+        auto advance = [&]() {
+            if (++s_i == n_q) { s_i = 0; ++s_li; }
+        };
+        if (total > 0) { stage_stats(0, s_li, s_i); advance(); }
+        if (total > 1) { stage_stats(1, s_li, s_i); advance(); }
         bool ok = true;
-        for (int t = 0; ok && t < n_q; ++t) {
-            if (!(ok = mbar_wait(&bars->dq_full, t & 1, abort_flag))) break;
+        int li = 0, i = 0, bh = item_bh(0);
+        for (int T = 0; ok && T < total; ++T) {
+            if (T > 0 && ++i == n_q) {
+                i = 0;
+                bh = item_bh(++li);
+            }
+            if (!(ok = mbar_wait(&bars->dq_full, T & 1, abort_flag))) break;
             tc_fence_after();
             uint32_t v[64];
             tmem_ld32(tmem + lane_off + Cfg::colDQ, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
             tmem_ld32(tmem + lane_off + Cfg::colDQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
             tmem_wait_ld();
-            stage_and_reduce(v, t * kTile);
+            stage_and_reduce(v, i * kTile, bh);
             tmem_ld32(tmem + lane_off + Cfg::colDQ + 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
             tmem_ld32(tmem + lane_off + Cfg::colDQ + 96, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&bars->dq_free);               // dQ^T columns may be overwritten now
-            // tile t's lse/D are no longer read (dS(t) is done): slot t&1 takes tile t+2
-            if (t + 2 < n_q) stage_stats(t + 2);
+            // tile T's lse/D are no longer read (dS(T) is done): slot T&1 takes tile T+2
+            if (T + 2 < total) {
+                stage_stats(T + 2, s_li, s_i);
+                advance();
+            }
             staging_reusable();
-            stage_and_reduce(v, t * kTile + 64);
+            stage_and_reduce(v, i * kTile + 64, bh);
             staging_reusable();
         }
         if (lane == 0) bulk_wait_all();                // every reduce-add has completed
@@ -530,16 +621,21 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
 }
 
-template <int D>
+template <int D, bool PERSIST>
 cudaError_t launch_main(const Bf16BwdArgs& a, cudaStream_t stream) {
-    using Cfg = BwdCfg<D>;
+    using Cfg = BwdCfg<D, PERSIST>;
     static_assert(Cfg::kSmemBytes <= 232448, "shared memory budget");
-    auto kern = bwd_main_kernel<D>;
+    auto kern = bwd_main_kernel<D, PERSIST>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
-    dim3 grid((a.Nk + kTile - 1) / kTile, a.BH, 1);
+    const int n_kt = (a.Nk + kTile - 1) / kTile;
+    dim3 grid(n_kt, a.BH, 1);
+    if (PERSIST) {
+        const long long items = (long long)n_kt * a.BH;
+        grid = dim3((unsigned)(items < a.sm_count ? items : a.sm_count), 1, 1);
+    }
     kern<<<grid, kThreads, Cfg::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.tm_dq_acc, a.lse, a.delta,
-                                                      a.dk, a.dv, a.dk_acc, a.dv_acc, a.Nq, a.Nk, a.scale);
+                                                      a.dk, a.dv, a.dk_acc, a.dv_acc, a.BH, a.Nq, a.Nk, a.scale);
     return cudaGetLastError();
 }
 
@@ -564,8 +660,13 @@ cudaError_t launch_bwd_bf16(const Bf16BwdArgs& a, cudaStream_t stream, unsigned 
     }
     cudaError_t e = cudaSuccess;
     if (phases & kBwdPhaseMain) {
-        e = (a.D == 64) ? launch_main<64>(a, stream) : (a.D == 128) ? launch_main<128>(a, stream)
-                                                                    : cudaErrorInvalidValue;
+        // D = 64 with few query tiles per key tile: persistent CTAs (two K/V
+        // buffers fit), whose next item's loads overlap the current item's end;
+        // otherwise one CTA per (head, key tile)
+        const bool persist = a.D == 64 && (a.Nq + kTile - 1) / kTile <= kBwdPersistMaxQTiles;
+        e = (a.D == 64) ? (persist ? launch_main<64, true>(a, stream) : launch_main<64, false>(a, stream))
+            : (a.D == 128) ? launch_main<128, false>(a, stream)
+                           : cudaErrorInvalidValue;
         if (e != cudaSuccess) return e;
     }
     if ((phases & kBwdPhaseFinal) && rows > 0) {

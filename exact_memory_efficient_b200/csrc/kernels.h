@@ -131,6 +131,7 @@ struct Bf16BwdArgs {
     float* dv_acc = nullptr;
     int BH, Nq, Nk, D;
     float scale;
+    int sm_count = 1;   // persistent grids (D = 64): at most one CTA per SM
 };
 // Phases of the backward, run in this order on one workspace.
 constexpr unsigned kBwdPhasePre = 1u;    // delta = rowsum(dO o O); dQ accumulator := 0

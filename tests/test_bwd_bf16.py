@@ -122,3 +122,23 @@ def test_dk_dv_deterministic():
     assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
     # dQ is accumulated with fp32 atomics: equal up to summation order
     assert torch.allclose(a[0].float(), b[0].float(), atol=1e-2)
+
+
+@pytest.mark.parametrize("B,H,Nq,Nk,D", [
+    (8, 16, 300, 700, 64),    # 768 (head, key tile) items: five or six per persistent CTA, ragged tails
+    (16, 16, 128, 77, 64),    # one query tile and one partial key tile per item, 256 items
+    (4, 20, 1000, 333, 64),   # eight query tiles per item, the longest loop that runs persistent
+    (1, 2, 1100, 260, 64),    # nine query tiles: one CTA per item
+])
+def test_persistent_items_backward(B, H, Nq, Nk, D):
+    """At D = 64 with at most 8 query tiles per key tile the backward runs persistent CTAs: the next
+    item's K, V load into the other buffer and its first S^T and P are formed before the current
+    item's epilogue has freed the dV, dK accumulators."""
+    w = custom(B, H, Nq, Nk, D, "bf16")
+    q, k, v, do = make_inputs(w, 19)
+    dq, dk, dv = gpu_fwd_bwd(q, k, v, do, w.scale)
+    rq, rk, rv, _, _ = oracle.attention_backward(to_f64(q), to_f64(k), to_f64(v), to_f64(do), w.scale)
+    what = f"{(B, H, Nq, Nk, D)}"
+    assert_close(to_np(dq), rq, *BF16_GRAD, what=f"dQ {what}")
+    assert_close(to_np(dk), rk, *BF16_GRAD, what=f"dK {what}")
+    assert_close(to_np(dv), rv, *BF16_GRAD, what=f"dV {what}")
