@@ -68,40 +68,81 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------ pre
 
-// One warp per query row: delta = sum_d dO * O (fp32), and dq_acc row := 0.
-__global__ void bwd_pre_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dO,
-                               float* __restrict__ delta, float* __restrict__ dq_acc, long long rows, int D) {
-    const long long row = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x / 32);
+// delta = sum_d dO * O (fp32) per query row, and the row of the fp32 dQ
+// accumulator := 0.  HBM-bound: each lane loads 16 bytes (8 bf16) of O and of
+// dO, D/8 lanes share a row, and a warp keeps kPreRows rows of loads in flight
+// before reducing (one 4-byte load per lane and row left too few bytes in
+// flight to stream HBM).
+constexpr int kPreRows = 4;   // row groups per warp per pass
+template <int D>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dO,
+                                                      float* __restrict__ delta, float* __restrict__ dq_acc,
+                                                      long long rows) {
+    constexpr int LPR = D / 8;          // lanes per row
+    constexpr int RPW = 32 / LPR;       // rows per warp and row group
     const int lane = threadIdx.x & 31;
-    if (row >= rows) return;
-    const uint16_t* orow = o + row * D;
-    const uint16_t* drow = dO + row * D;
-    float acc = 0.f;
-    for (int d = 2 * lane; d < D; d += 64) {
-        const uint32_t ov = *reinterpret_cast<const uint32_t*>(orow + d);
-        const uint32_t dv = *reinterpret_cast<const uint32_t*>(drow + d);
-        acc = fmaf(__uint_as_float(ov << 16), __uint_as_float(dv << 16), acc);
-        acc = fmaf(__uint_as_float(ov & 0xffff0000u), __uint_as_float(dv & 0xffff0000u), acc);
+    const int sub = lane / LPR, l = lane % LPR;
+    const long long warp_g = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const long long row0 = warp_g * (RPW * kPreRows) + sub;
+    uint4 ov[kPreRows], dv[kPreRows];
+#pragma unroll
+    for (int u = 0; u < kPreRows; ++u) {
+        const long long r = row0 + u * RPW;
+        if (r < rows) {
+            ov[u] = *reinterpret_cast<const uint4*>(o + r * D + 8 * l);
+            dv[u] = *reinterpret_cast<const uint4*>(dO + r * D + 8 * l);
+        } else {
+            ov[u] = dv[u] = make_uint4(0, 0, 0, 0);
+        }
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) delta[row] = acc;
-    if (dq_acc == nullptr) return;   // accumulating callers own (and keep) their dQ accumulator
-    float4* z = reinterpret_cast<float4*>(dq_acc + row * D);
-    for (int c = lane; c < D / 4; c += 32) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < kPreRows; ++u) {
+        const uint32_t ow[4] = {ov[u].x, ov[u].y, ov[u].z, ov[u].w};
+        const uint32_t dw[4] = {dv[u].x, dv[u].y, dv[u].z, dv[u].w};
+        float acc = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            acc = fmaf(__uint_as_float(ow[c] << 16), __uint_as_float(dw[c] << 16), acc);
+            acc = fmaf(__uint_as_float(ow[c] & 0xffff0000u), __uint_as_float(dw[c] & 0xffff0000u), acc);
+        }
+#pragma unroll
+        for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        const long long r = row0 + u * RPW;
+        if (r < rows) {
+            if (l == 0) delta[r] = acc;
+            if (dq_acc != nullptr) {   // accumulating callers own (and keep) their dQ accumulator
+                float4* z = reinterpret_cast<float4*>(dq_acc + r * D) + 2 * l;
+                z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+                z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+    }
 }
 
 // ------------------------------------------------------------- finalise
 
-__global__ void bwd_dq_final_kernel(const float* __restrict__ dq_acc, uint16_t* __restrict__ dq,
-                                    long long n4, float scale) {
-    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= n4) return;
-    const float4 a = reinterpret_cast<const float4*>(dq_acc)[i];
-    uint2 r;
-    r.x = pack_bf16x2(a.x * scale, a.y * scale);
-    r.y = pack_bf16x2(a.z * scale, a.w * scale);
-    reinterpret_cast<uint2*>(dq)[i] = r;
+// dq = bf16(scale * dQacc): each thread converts kFinalVecs float4 groups, all
+// loads issued before the first store.
+constexpr int kFinalVecs = 4;
+__global__ void __launch_bounds__(256) bwd_dq_final_kernel(const float* __restrict__ dq_acc, uint16_t* __restrict__ dq,
+                                                           long long n4, float scale) {
+    const long long base = (long long)blockIdx.x * blockDim.x * kFinalVecs + threadIdx.x;
+    float4 a[kFinalVecs];
+#pragma unroll
+    for (int u = 0; u < kFinalVecs; ++u) {
+        const long long i = base + (long long)u * blockDim.x;
+        a[u] = i < n4 ? reinterpret_cast<const float4*>(dq_acc)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kFinalVecs; ++u) {
+        const long long i = base + (long long)u * blockDim.x;
+        if (i < n4) {
+            uint2 r;
+            r.x = pack_bf16x2(a[u].x * scale, a[u].y * scale);
+            r.y = pack_bf16x2(a[u].z * scale, a[u].w * scale);
+            reinterpret_cast<uint2*>(dq)[i] = r;
+        }
+    }
 }
 
 // fp32 accumulator -> output dtype: out = mul * acc (bf16 round to nearest even, or fp32)
@@ -652,9 +693,15 @@ cudaError_t launch_accum_convert(const float* acc, void* out, long long n, float
 cudaError_t launch_bwd_bf16(const Bf16BwdArgs& a, cudaStream_t stream, unsigned phases) {
     const long long rows = (long long)a.BH * a.Nq;
     if ((phases & kBwdPhasePre) && rows > 0) {
-        const int warps = 8;
-        const long long blocks = (rows + warps - 1) / warps;
-        bwd_pre_kernel<<<(unsigned)blocks, 32 * warps, 0, stream>>>(a.o, a.dO, a.delta, a.dq_acc, rows, a.D);
+        const long long rows_per_warp = (long long)(32 / (a.D / 8)) * kPreRows;
+        const long long warps = (rows + rows_per_warp - 1) / rows_per_warp;
+        const unsigned blocks = (unsigned)((warps + 7) / 8);
+        if (a.D == 64)
+            bwd_pre_kernel<64><<<blocks, 256, 0, stream>>>(a.o, a.dO, a.delta, a.dq_acc, rows);
+        else if (a.D == 128)
+            bwd_pre_kernel<128><<<blocks, 256, 0, stream>>>(a.o, a.dO, a.delta, a.dq_acc, rows);
+        else
+            return cudaErrorInvalidValue;
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -672,7 +719,9 @@ cudaError_t launch_bwd_bf16(const Bf16BwdArgs& a, cudaStream_t stream, unsigned 
     if ((phases & kBwdPhaseFinal) && rows > 0) {
         const long long n4 = rows * a.D / 4;
         const int tpb = 256;
-        bwd_dq_final_kernel<<<(unsigned)((n4 + tpb - 1) / tpb), tpb, 0, stream>>>(a.dq_acc, a.dq, n4, a.scale);
+        const long long per_block = (long long)tpb * kFinalVecs;
+        bwd_dq_final_kernel<<<(unsigned)((n4 + per_block - 1) / per_block), tpb, 0, stream>>>(a.dq_acc, a.dq, n4,
+                                                                                              a.scale);
         e = cudaGetLastError();
     }
     return e;
