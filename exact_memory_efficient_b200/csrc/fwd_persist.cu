@@ -9,24 +9,36 @@
 // Why: with a few key tiles per (head, query-tile pair) the one-CTA-per-item
 // forward spends much of each CTA on its fixed cost (barriers, TMEM, the Q
 // load) and on filling and draining its pipeline.  Here a grid of at most one
-// CTA per SM walks the items in a fixed order (CTA c takes items c, c + G,
-// c + 2G, ...), keeping its barriers, TMEM and K/V ring: the next item's Q is
-// loaded as soon as the current item's last S has been issued, and its first
-// S and the producer's K/V loads overlap the current item's epilogue.
+// CTA per SM walks a fixed list of items (CTA c takes items c, c + G, c + 2G,
+// ...), keeping its barriers, TMEM and K/V ring: the next item's Q is loaded
+// as soon as the current item's last S has been issued, and its first S and
+// the producer's K/V loads overlap the current item's epilogue.
+//
+// Items.  A pair item is one (head, query-tile pair): slot t holds query tile
+// t and every key tile.  When the pair items do not fill the last round of
+// the grid (n pairs over G CTAs leave r = n mod G of them for a last round in
+// which most CTAs would idle), the last r pairs are listed instead as 2r
+// single items of one query tile each, provided 2r <= G: the two slots of a
+// single item run the recurrence for the same rows over alternate key tiles
+// (slot t takes tiles t, t+2, ...) and slot 0 folds slot 1's summary in with
+// the two-block formulas at the end, so the last round takes about half the
+// time of a pair round.
 //
 // Roles (320 threads) as in fwd_bf16.cu's two-tile path:
-//   warp 0       TMEM allocator, then TMA producer (Q pair per item; K_0, V_0,
+//   warp 0       TMEM allocator, then TMA producer (Q tiles per item; K_0, V_0,
 //                K_1, V_1, ... of each item through the ring; no multicast)
 //   warp 1       MMA issuer (one thread)
-//   warps 2-5    softmax / epilogue of query tile 0, warps 6-9 of tile 1
-// Phases of the per-key-tile barriers run on across items (the parity is
-// that of the CTA's running key-tile count).  Per item, q_empty (Q may be
-// replaced), o_final (O complete) and o_free[t] (tile t's O has been read by
-// the epilogue, so the next item's first P V may overwrite it) complete once.
+//   warps 2-5    softmax / epilogue of slot 0, warps 6-9 of slot 1
+// Phases of the per-key-tile barriers run on across items (the parity is that
+// of the slot's running key-tile count).  Per item, q_empty (Q may be
+// replaced), o_final (O complete) and o_free[t] (slot t's O has been read by
+// the epilogue, so the next item's first P V may overwrite it) complete once;
+// merge_ready (slot 1's row summaries are in shared memory) once per single
+// item.
 // TMEM: S_0 [0,128) S_1 [128,256) O_0 [256,256+D) O_1 [384,384+D).
 //
-// Used for bf16 Q/K/V when every CTA would hold two full query tiles (Nq a
-// multiple of 256), the keys are not split, and the key range is short.
+// Used for bf16 Q/K/V when Nq is a multiple of 256, the keys are not split,
+// and the key range is short.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -65,27 +77,52 @@ struct PersistBarriers {
     uint64_t p_ready[2];
     uint64_t o_final;
     uint64_t o_free[2];
+    uint64_t merge_ready;
     uint64_t drain;
     unsigned tmem_base;
     int abort_flag;
 };
 
-template <int D>
+// Item `item` of the list: the first n_pair_items are (head, query-tile pair)
+// items in head-major order; the rest are the query tiles of the remaining
+// pairs, one per item, in the same order.
+struct PersistItem {
+    int bh;
+    int q0;       // first query row
+    bool single;  // one query tile (both slots on its rows)
+};
+
+__device__ __forceinline__ PersistItem persist_item(int item, int pairs, int n_pair_items) {
+    PersistItem it;
+    it.single = item >= n_pair_items;
+    const int p = it.single ? n_pair_items + ((item - n_pair_items) >> 1) : item;   // pair index
+    it.bh = p / pairs;
+    it.q0 = (p - it.bh * pairs) * (2 * kTileP) + (it.single ? ((item - n_pair_items) & 1) * kTileP : 0);
+    return it;
+}
+
+// SINGLES: the item list may hold single query tiles (a launch whose list has
+// none uses the instantiation without their code paths).
+template <int D, bool SINGLES>
 __global__ void __launch_bounds__(kThreadsP, 1)
 fwd_persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ o, float* __restrict__ lse,
-                   int BH, int Nq, int Nk, float scale) {
+                   int Nq, int Nk, float scale, int n_pair_items, int n_items) {
     using Cfg = PersistCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* sQ = smem;
     uint8_t* sRing = smem + 2 * Cfg::kQBytes;
+    // Both slots' (m_ref, l) per row of a single item go to the second Q tile's
+    // buffer: single items come after every pair item of the list and load only
+    // the first Q tile, so once a CTA reaches its first single item nothing
+    // writes or reads that buffer any more.
+    float* sMerge = reinterpret_cast<float*>(smem + Cfg::kQBytes);
     PersistBarriers* bars = reinterpret_cast<PersistBarriers*>(smem + Cfg::kSmemData);
 
     const unsigned warp = warp_id();
     const unsigned lane = lane_id();
     const int pairs = Nq / (2 * kTileP);             // query-tile pairs per head
-    const int n_items = BH * pairs;
     const int n_kv = (Nk + kTileP - 1) / kTileP;
     // this CTA's items: blockIdx.x, blockIdx.x + gridDim.x, ...
     const int first = (int)blockIdx.x;
@@ -106,6 +143,7 @@ fwd_persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_init(&bars->o_free[t], 128);
         }
         mbar_init(&bars->o_final, 1);
+        mbar_init(&bars->merge_ready, 256);
         mbar_init(&bars->drain, 1);
         bars->abort_flag = 0;
         fence_mbar_init();
@@ -127,18 +165,17 @@ fwd_persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
             int c_glob = 0;       // ring tiles issued so far (all items)
-            int q_issued = 0;     // items whose Q pair has been requested
+            int q_issued = 0;     // items whose Q has been requested
             bool ok = true;
             for (int li = 0; ok && li < my_items; ++li) {
-                const int item = first + li * stride;
-                const int bh = item / pairs;
-                const int m0 = (item - bh * pairs) * (2 * kTileP);
+                const PersistItem itm = persist_item(first + li * stride, pairs, n_pair_items);
+                const int n_qt = itm.single ? 1 : 2;
                 if (li > 0 && !(ok = mbar_wait(&bars->q_empty, (li - 1) & 1, abort_flag))) break;
-                mbar_arrive_expect_tx(&bars->q_full, 2 * Cfg::kQBytes);
-                for (int t = 0; t < 2; ++t)
+                mbar_arrive_expect_tx(&bars->q_full, n_qt * Cfg::kQBytes);
+                for (int t = 0; t < n_qt; ++t)
                     for (int b = 0; b < D / 64; ++b)
                         tma_load_3d(sQ + t * Cfg::kQBytes + b * Cfg::kBoxBytes, &tm_q, &bars->q_full, b * 64,
-                                    m0 + t * kTileP, bh);
+                                    itm.q0 + t * kTileP, itm.bh);
                 q_issued = li + 1;
                 for (int c = 0; c < 2 * n_kv; ++c, ++c_glob) {
                     const int s = c_glob % Cfg::kStages;
@@ -149,7 +186,7 @@ fwd_persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     mbar_arrive_expect_tx(&bars->full[s], Cfg::kTileBytes);
                     for (int b = 0; b < D / 64; ++b)
                         tma_load_3d(sRing + s * Cfg::kTileBytes + b * Cfg::kBoxBytes, tm, &bars->full[s], b * 64,
-                                    (c >> 1) * kTileP, bh);
+                                    (c >> 1) * kTileP, itm.bh);
                 }
             }
             // never leave with copies in flight
@@ -198,43 +235,88 @@ fwd_persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 return true;
             };
             bool ok = true;
-            int kt = 0;   // key tiles completed by this CTA (all items): phase of s_full / p_half / p_ready
+            // key tiles completed by each slot (all items): phase of s_full / p_half / p_ready
+            // (scalars, not an array indexed by the slot, so that they stay in registers)
+            int cnt0 = 0, cnt1 = 0;
             for (int li = 0; ok && li < my_items; ++li) {
+                const bool single = SINGLES && first + li * stride >= n_pair_items;
+                // after a single item both slots read both O: the first P V of
+                // either slot waits for both epilogues
+                const bool prev_single = SINGLES && li > 0 && first + (li - 1) * stride >= n_pair_items;
                 if (!(ok = mbar_wait(&bars->q_full, li & 1, abort_flag))) break;
                 uint32_t k_off = 0;
                 int k_stage = 0;
-                if (!(ok = next_tile(k_off, k_stage))) break;
-                tc_fence_after();
-                issue_s(tS0, q_lo0, k_off);
-                mma_commit(&bars->s_full[0]);
-                issue_s(tS1, q_lo1, k_off);
-                mma_commit(&bars->s_full[1]);
-                mma_commit(&bars->empty[k_stage]);
-                if (n_kv == 1) mma_commit(&bars->q_empty);      // Q read by its last S
-                for (int j = 0; ok && j < n_kv; ++j, ++kt) {
-                    const bool more = (j + 1 < n_kv);
-                    const unsigned acc0 = j > 0 ? 1u : 0u;
-                    uint32_t v_off = 0;
-                    int v_stage = 0;
-                    if (!(ok = next_tile(v_off, v_stage))) break;
-                    // the first P V of an item overwrites O: the epilogue of the
-                    // previous item must have read it
-                    if (j == 0 && li > 0 && !(ok = mbar_wait(&bars->o_free[0], (li - 1) & 1, abort_flag))) break;
-                    if (!(ok = pv_halves(0, kt & 1, v_off, acc0))) break;
-                    if (more) {
+                if (single) {
+                    // both slots on query tile 0 over alternate key tiles; the ring
+                    // is still taken in the producer's order K_0, V_0, K_1, V_1, ...
+                    // and a slot's V tile is held until its P is ready
+                    uint32_t v_off0 = 0, v_off1 = 0;
+                    int v_stage0 = 0, v_stage1 = 0;
+                    for (int t = 0; ok && t < 2 && t < n_kv; ++t) {
                         if (!(ok = next_tile(k_off, k_stage))) break;
                         tc_fence_after();
-                        issue_s(tS0, q_lo0, k_off);
-                        mma_commit(&bars->s_full[0]);
-                    }
-                    if (j == 0 && li > 0 && !(ok = mbar_wait(&bars->o_free[1], (li - 1) & 1, abort_flag))) break;
-                    if (!(ok = pv_halves(1, kt & 1, v_off, acc0))) break;
-                    mma_commit(&bars->empty[v_stage]);
-                    if (more) {
-                        issue_s(tS1, q_lo1, k_off);
-                        mma_commit(&bars->s_full[1]);
+                        issue_s(t ? tS1 : tS0, q_lo0, k_off);
+                        mma_commit(&bars->s_full[t]);
                         mma_commit(&bars->empty[k_stage]);
-                        if (j + 2 == n_kv) mma_commit(&bars->q_empty);   // Q read by its last S
+                        if (t + 1 == n_kv) mma_commit(&bars->q_empty);   // Q read by its last S
+                        ok = t ? next_tile(v_off1, v_stage1) : next_tile(v_off0, v_stage0);
+                    }
+                    for (int j = 0; ok && j < n_kv; ++j) {
+                        const int t = j & 1;
+                        // the first P V of a slot overwrites its O: the epilogue of
+                        // the previous item must have read it
+                        if (j < 2 && li > 0 && !(ok = mbar_wait(&bars->o_free[t], (li - 1) & 1, abort_flag))) break;
+                        if (j == 0 && prev_single && !(ok = mbar_wait(&bars->o_free[1], (li - 1) & 1, abort_flag))) break;
+                        if (!(ok = pv_halves(t, (t ? cnt1 : cnt0) & 1, t ? v_off1 : v_off0, j >= 2 ? 1u : 0u))) break;
+                        if (t) ++cnt1; else ++cnt0;
+                        mma_commit(&bars->empty[t ? v_stage1 : v_stage0]);
+                        if (j + 2 < n_kv) {
+                            if (!(ok = next_tile(k_off, k_stage))) break;
+                            tc_fence_after();
+                            issue_s(t ? tS1 : tS0, q_lo0, k_off);
+                            mma_commit(&bars->s_full[t]);
+                            mma_commit(&bars->empty[k_stage]);
+                            if (j + 3 == n_kv) mma_commit(&bars->q_empty);
+                            ok = t ? next_tile(v_off1, v_stage1) : next_tile(v_off0, v_stage0);
+                        }
+                    }
+                } else {
+                    if (!(ok = next_tile(k_off, k_stage))) break;
+                    tc_fence_after();
+                    issue_s(tS0, q_lo0, k_off);
+                    mma_commit(&bars->s_full[0]);
+                    issue_s(tS1, q_lo1, k_off);
+                    mma_commit(&bars->s_full[1]);
+                    mma_commit(&bars->empty[k_stage]);
+                    if (n_kv == 1) mma_commit(&bars->q_empty);      // Q read by its last S
+                    for (int j = 0; ok && j < n_kv; ++j) {
+                        const bool more = (j + 1 < n_kv);
+                        const unsigned acc0 = j > 0 ? 1u : 0u;
+                        uint32_t v_off = 0;
+                        int v_stage = 0;
+                        if (!(ok = next_tile(v_off, v_stage))) break;
+                        // the first P V of an item overwrites O: the epilogue of the
+                        // previous item must have read it
+                        if (j == 0 && li > 0 && !(ok = mbar_wait(&bars->o_free[0], (li - 1) & 1, abort_flag))) break;
+                        if (j == 0 && prev_single && !(ok = mbar_wait(&bars->o_free[1], (li - 1) & 1, abort_flag))) break;
+                        if (!(ok = pv_halves(0, cnt0 & 1, v_off, acc0))) break;
+                        ++cnt0;
+                        if (more) {
+                            if (!(ok = next_tile(k_off, k_stage))) break;
+                            tc_fence_after();
+                            issue_s(tS0, q_lo0, k_off);
+                            mma_commit(&bars->s_full[0]);
+                        }
+                        if (j == 0 && li > 0 && !(ok = mbar_wait(&bars->o_free[1], (li - 1) & 1, abort_flag))) break;
+                        if (!(ok = pv_halves(1, cnt1 & 1, v_off, acc0))) break;
+                        ++cnt1;
+                        mma_commit(&bars->empty[v_stage]);
+                        if (more) {
+                            issue_s(tS1, q_lo1, k_off);
+                            mma_commit(&bars->s_full[1]);
+                            mma_commit(&bars->empty[k_stage]);
+                            if (j + 2 == n_kv) mma_commit(&bars->q_empty);   // Q read by its last S
+                        }
                     }
                 }
                 if (ok) mma_commit(&bars->o_final);
@@ -252,21 +334,24 @@ fwd_persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const unsigned tO = tmem + lane_off + (t ? 384u : 256u);
         const float c_log2 = fabsf(scale) * kLog2eP;   // S carries the sign (A negated)
         bool ok = true;
-        int kt = 0;
+        int kt = 0;         // key tiles completed by this slot (all items)
+        int n_single = 0;   // single items completed by this CTA
         for (int li = 0; ok && li < my_items; ++li) {
             const int item = first + li * stride;
-            const int bh = item / pairs;
-            const int row = (item - bh * pairs) * (2 * kTileP) + t * kTileP + r;
+            const bool single = SINGLES && item >= n_pair_items;
+            // a pair item's slot t owns query tile t and every key tile; a single
+            // item's slots own its one tile and key tiles t, t+2, ...
+            const int n_mine = single ? (n_kv + 1 - t) / 2 : n_kv;
             float m_ref = -INFINITY;
             float l = 0.f;
-            for (int it = 0; it < n_kv; ++it, ++kt) {
+            for (int it = 0; it < n_mine; ++it, ++kt) {
+                const int nvalid = Nk - (single ? 2 * it + t : it) * kTileP;   // keys from this tile on
                 if (!(ok = mbar_wait(&bars->s_full[t], kt & 1, abort_flag))) break;
                 tc_fence_after();
                 uint32_t sr[kTileP];
 #pragma unroll
                 for (int c0 = 0; c0 < kTileP; c0 += 32) tmem_ld32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(&sr[c0]));
                 tmem_wait_ld();
-                const int nvalid = Nk - it * kTileP;
                 if (nvalid < kTileP) {
 #pragma unroll
                     for (int c = 0; c < kTileP; ++c)
@@ -315,8 +400,8 @@ fwd_persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 l += ((rsa[0] + rsa[1]) + (rsa[2] + rsa[3])) + ((rsa[4] + rsa[5]) + (rsa[6] + rsa[7]));
                 if (rescale) {
-                    // P V of the previous key tile has completed (it was issued
-                    // before S of this one, whose commit was waited on)
+                    // P V of this slot's previous key tile has completed (it was
+                    // issued before S of this one, whose commit was waited on)
 #pragma unroll
                     for (int c0 = 0; c0 < D; c0 += 32) {
                         uint32_t ov[32];
@@ -332,25 +417,70 @@ fwd_persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 if (rescale) mbar_arrive(&bars->p_half[t]);
                 mbar_arrive(&bars->p_ready[t]);
             }
-            if (!ok || !(ok = mbar_wait(&bars->o_final, li & 1, abort_flag))) break;
+            if (!ok) break;
+            // A single item's slots fold their summaries of the same rows
+            // together with the two-block formulas and each writes half of the
+            // head dims, reading both slots' O (slot 1 is empty when the item
+            // has one key tile; its summary is then m = -inf, l = 0).
+            const bool with1 = single && n_kv >= 2;
+            // (the item's rows are found while the last P V is still running)
+            const PersistItem itm = persist_item(item, pairs, n_pair_items);
+            const int row = itm.q0 + (single ? 0 : t * kTileP) + r;
+            float w0 = 1.f, w1 = 0.f, M = m_ref, L = l;
+            if (single) {
+                // the other slot has read the previous single item's summaries:
+                // its o_free of the previous item completed after its epilogue
+                if (li > 0 && !(ok = mbar_wait(&bars->o_free[t ^ 1], (li - 1) & 1, abort_flag))) break;
+                sMerge[2 * (t * kTileP + r)] = m_ref;
+                sMerge[2 * (t * kTileP + r) + 1] = l;
+                mbar_arrive(&bars->merge_ready);
+                if (!(ok = mbar_wait(&bars->merge_ready, n_single & 1, abort_flag))) break;
+                ++n_single;
+                const float m_o = sMerge[2 * ((t ^ 1) * kTileP + r)];
+                const float l_o = sMerge[2 * ((t ^ 1) * kTileP + r) + 1];
+                M = fmaxf(m_ref, m_o);
+                const float w_self = ex2_approx(m_ref - M), w_oth = ex2_approx(m_o - M);
+                L = w_self * l + w_oth * l_o;
+                w0 = t ? w_oth : w_self;
+                w1 = t ? w_self : w_oth;
+            }
+            if (!(ok = mbar_wait(&bars->o_final, li & 1, abort_flag))) break;
             tc_fence_after();
-            const float inv_l = 1.f / l;
-            uint16_t* orow = o + ((size_t)bh * Nq + row) * D;
+            const float inv_l = 1.f / L;
+            const float s0 = w0 * inv_l, s1 = w1 * inv_l;
+            // pair item: slot t writes every head dim of its own O; single item:
+            // slot t writes dims [t D/2, (t+1) D/2) of O_0 s0 + O_1 s1
+            const int c_begin = single ? t * (D / 2) : 0;
+            const int n_chunks = single ? D / 32 : D / 16;
+            const unsigned tOa = single ? tmem + lane_off + 256u : tO;
+            const unsigned tOb = tmem + lane_off + 384u;
+            uint16_t* orow = o + ((size_t)itm.bh * Nq + row) * D;
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 16) {
-                uint32_t a0[16];
-                tmem_ld16(tO + c0, a0);
+            for (int k = 0; k < D / 16; ++k) {
+                if (k >= n_chunks) break;
+                const int c0 = c_begin + 16 * k;
+                uint32_t a[16];
+                float f[16];
+                tmem_ld16(tOa + c0, a);
                 tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(a[i]) * s0;
+                if (with1) {
+                    tmem_ld16(tOb + c0, a);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) f[i] = fmaf(__uint_as_float(a[i]), s1, f[i]);
+                }
                 uint32_t packed[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    packed[i] = pack_bf16x2(__uint_as_float(a0[2 * i]) * inv_l, __uint_as_float(a0[2 * i + 1]) * inv_l);
+                for (int i = 0; i < 8; ++i) packed[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
                 uint4* dst = reinterpret_cast<uint4*>(orow + c0);
                 dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
                 dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
             }
-            lse[(size_t)bh * Nq + row] = (m_ref + __log2f(l)) * kLn2P;
-            // this tile's O has been read: the next item's first P V may overwrite it
+            if (!single || t == 0) lse[(size_t)itm.bh * Nq + row] = (M + __log2f(L)) * kLn2P;
+            // this slot's reads of O are done (a single item's O_0 and O_1 are
+            // both read by both slots: the next item's first P V waits for both)
             tc_fence_before();
             mbar_arrive(&bars->o_free[t]);
         }
@@ -364,21 +494,43 @@ fwd_persist_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
 }
 
-template <int D>
-cudaError_t launch_persist(const Bf16FwdArgs& a, int sm_count, cudaStream_t stream) {
+template <int D, bool SINGLES>
+cudaError_t launch_persist_list(const Bf16FwdArgs& a, const PersistSchedule& sch, cudaStream_t stream) {
     using Cfg = PersistCfg<D>;
-    auto kern = fwd_persist_kernel<D>;
+    auto kern = fwd_persist_kernel<D, SINGLES>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
-    const long long items = (long long)a.BH * (a.Nq / (2 * kTileP));
-    const long long grid = items < sm_count ? items : sm_count;
-    if (grid <= 0) return cudaSuccess;
-    kern<<<(unsigned)grid, kThreadsP, Cfg::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.o, a.lse, a.BH, a.Nq,
-                                                                   a.Nk, a.scale);
+    kern<<<(unsigned)sch.grid, kThreadsP, Cfg::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.o, a.lse, a.Nq, a.Nk,
+                                                                       a.scale, (int)sch.n_pair_items,
+                                                                       (int)sch.n_items);
     return cudaGetLastError();
 }
 
+template <int D>
+cudaError_t launch_persist(const Bf16FwdArgs& a, int sm_count, cudaStream_t stream) {
+    const PersistSchedule sch = fwd_persist_schedule((long long)a.BH * (a.Nq / (2 * kTileP)), sm_count);
+    if (sch.grid <= 0) return cudaSuccess;
+    return sch.n_items > sch.n_pair_items ? launch_persist_list<D, true>(a, sch, stream)
+                                          : launch_persist_list<D, false>(a, sch, stream);
+}
+
 }  // namespace
+
+PersistSchedule fwd_persist_schedule(long long n_pairs, int sm_count) {
+    PersistSchedule s;
+    s.n_pair_items = n_pairs;
+    s.n_items = n_pairs;
+    s.grid = n_pairs < sm_count ? n_pairs : sm_count;
+    if (n_pairs <= 0 || sm_count <= 0) return s;
+    const long long rounds = n_pairs / sm_count;
+    const long long rest = n_pairs - rounds * sm_count;   // pairs of a partial last round
+    if (rest > 0 && 2 * rest <= sm_count) {
+        s.n_pair_items = n_pairs - rest;
+        s.n_items = n_pairs + rest;
+        s.grid = rounds > 0 ? sm_count : 2 * rest;
+    }
+    return s;
+}
 
 bool fwd_persist_applies(int D, bool fp8_qk, int Nq, int Nk, int chunks) {
     return (D == 64 || D == 128) && !fp8_qk && chunks <= 1 && Nq >= 2 * kTileP && Nq % (2 * kTileP) == 0 &&
@@ -387,6 +539,7 @@ bool fwd_persist_applies(int D, bool fp8_qk, int Nq, int Nk, int chunks) {
 
 cudaError_t launch_fwd_persist(const Bf16FwdArgs& a, int sm_count, cudaStream_t stream) {
     if (!fwd_persist_applies(a.D, a.fp8_qk, a.Nq, a.Nk, a.chunks)) return cudaErrorInvalidValue;
+    if ((long long)a.BH * (a.Nq / (2 * kTileP)) * 2 > 0x7fffffffLL) return cudaErrorInvalidValue;
     return a.D == 64 ? launch_persist<64>(a, sm_count, stream) : launch_persist<128>(a, sm_count, stream);
 }
 

@@ -108,6 +108,14 @@ constexpr int kFwdPersistMaxKeys128 = 2048;
 constexpr int kFwdPersistMaxKeys64 = 4096;
 bool fwd_persist_applies(int D, bool fp8_qk, int Nq, int Nk, int chunks);
 cudaError_t launch_fwd_persist(const Bf16FwdArgs& a, int sm_count, cudaStream_t stream);
+// Item list of the persistent forward for n_pairs (head, query-tile pair)
+// items on sm_count SMs: the first n_pair_items are pairs; when the pairs of a
+// partial last round number r with 2r <= sm_count, those r pairs are listed as
+// 2r single query tiles instead (n_items = n_pairs + r).  grid = CTAs launched.
+struct PersistSchedule {
+    long long n_pair_items, n_items, grid;
+};
+PersistSchedule fwd_persist_schedule(long long n_pairs, int sm_count);
 // Clusters of `cluster` CTAs of the tensor-core forward instantiation that a
 // launch with these D, operand type and Nq uses that can be resident at once
 // (cudaOccupancyMaxActiveClusters); 0 on failure.

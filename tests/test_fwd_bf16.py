@@ -237,10 +237,19 @@ def test_negative_scale(B, H, Nq, Nk, D):
     (4, 20, 768, 333, 128),   # three query-tile pairs per head, three key tiles
     (2, 3, 256, 4096, 64),    # the longest key range that takes the persistent CTAs at D = 64
     (3, 5, 512, 2048, 128),   # and at D = 128
+    # Item lists with single query tiles (the two slots of a CTA split the keys) for the pairs
+    # of a partial last round, on a part with 148 SMs:
+    (16, 16, 512, 333, 64),   # 512 pairs: three full rounds, the last 68 pairs as 136 single tiles (3 key tiles: 2 + 1)
+    (16, 16, 512, 700, 128),  # the same at D = 128 with 6 key tiles (the last ragged)
+    (2, 37, 256, 500, 64),    # 74 pairs: all as 148 single tiles, one round
+    (1, 16, 1024, 1024, 128), # 64 pairs: 128 single tiles with 8 key tiles each
+    (1, 16, 256, 256, 128),   # 16 pairs: 32 single tiles with 2 key tiles each
 ])
 def test_persistent_items_full(B, H, Nq, Nk, D):
     """Short key ranges with Nq a multiple of 256: CTAs walk several (head, tile pair) items,
-    reusing their barriers, TMEM and K/V ring from one item to the next."""
+    reusing their barriers, TMEM and K/V ring from one item to the next.  Where the pairs would
+    leave most CTAs idle in a last round, those pairs run as single query tiles whose two
+    slots take alternate key tiles and merge their summaries with the two-block formulas."""
     w = custom(B, H, Nq, Nk, D, "bf16", backward=False)
     q, k, v, _ = make_inputs(w, 16)
     full_check(q, k, v, w.scale, f"persistent {(B, H, Nq, Nk, D)}")
