@@ -208,7 +208,7 @@ mea_status_t tc_forward(const void* q, const void* k, const void* v, void* o, fl
         a.chunk_len = (int)round_up((size_t)((Nk + chunks - 1) / chunks), 128);
         if ((long long)((Nq + 255) / 256) * chunks > 0x7fffffffLL) return MEA_ERR_UNSUPPORTED;
     }
-    if (mea::fwd_persist_applies(D, fp8, Nq, Nk, a.chunks))
+    if (mea::fwd_persist_applies(D, fp8, BH, Nq, Nk, a.chunks, dev->sm_count))
         return cuda_status(mea::launch_fwd_persist(a, dev->sm_count, s), "fwd_persist launch");
     return cuda_status(mea::launch_fwd_bf16(a, s), "fwd_bf16 launch");
 }

@@ -532,13 +532,21 @@ PersistSchedule fwd_persist_schedule(long long n_pairs, int sm_count) {
     return s;
 }
 
-bool fwd_persist_applies(int D, bool fp8_qk, int Nq, int Nk, int chunks) {
-    return (D == 64 || D == 128) && !fp8_qk && chunks <= 1 && Nq >= 2 * kTileP && Nq % (2 * kTileP) == 0 &&
-           Nk >= 1 && Nk <= (D == 64 ? kFwdPersistMaxKeys64 : kFwdPersistMaxKeys128);
+bool fwd_persist_applies(int D, bool fp8_qk, int BH, int Nq, int Nk, int chunks, int sm_count) {
+    if (!((D == 64 || D == 128) && !fp8_qk && chunks <= 1 && Nq >= 2 * kTileP && Nq % (2 * kTileP) == 0 && Nk >= 1))
+        return false;
+    const int max_keys = D == 64 ? kFwdPersistMaxKeys64 : kFwdPersistMaxKeys128;
+    if (Nk <= max_keys) return true;
+    // longer key ranges amortise a CTA's fixed cost by themselves, but where
+    // the pairs leave a partial last round that single tiles can halve, the
+    // item list still gains up to twice the key limit
+    if (Nk > 2 * max_keys) return false;
+    const PersistSchedule s = fwd_persist_schedule((long long)BH * (Nq / (2 * kTileP)), sm_count);
+    return s.n_items > s.n_pair_items;
 }
 
 cudaError_t launch_fwd_persist(const Bf16FwdArgs& a, int sm_count, cudaStream_t stream) {
-    if (!fwd_persist_applies(a.D, a.fp8_qk, a.Nq, a.Nk, a.chunks)) return cudaErrorInvalidValue;
+    if (!fwd_persist_applies(a.D, a.fp8_qk, a.BH, a.Nq, a.Nk, a.chunks, sm_count)) return cudaErrorInvalidValue;
     if ((long long)a.BH * (a.Nq / (2 * kTileP)) * 2 > 0x7fffffffLL) return cudaErrorInvalidValue;
     return a.D == 64 ? launch_persist<64>(a, sm_count, stream) : launch_persist<128>(a, sm_count, stream);
 }

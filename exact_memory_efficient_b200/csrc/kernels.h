@@ -103,10 +103,11 @@ cudaError_t launch_fwd_bf16(const Bf16FwdArgs& a, cudaStream_t stream);
 // SM walks the (head, query-tile pair) items, for bf16 Q/K/V at D = 64 or 128
 // when every item holds two full query tiles (Nq a multiple of 256), the keys
 // are not split and the key range is short: Nk <= 2048 at D = 128, 4096 at
-// D = 64 (longer ranges amortise a CTA's fixed cost by themselves).
+// D = 64 (longer ranges amortise a CTA's fixed cost by themselves), or up to
+// twice that when the item list has single query tiles (fwd_persist_schedule).
 constexpr int kFwdPersistMaxKeys128 = 2048;
 constexpr int kFwdPersistMaxKeys64 = 4096;
-bool fwd_persist_applies(int D, bool fp8_qk, int Nq, int Nk, int chunks);
+bool fwd_persist_applies(int D, bool fp8_qk, int BH, int Nq, int Nk, int chunks, int sm_count);
 cudaError_t launch_fwd_persist(const Bf16FwdArgs& a, int sm_count, cudaStream_t stream);
 // Item list of the persistent forward for n_pairs (head, query-tile pair)
 // items on sm_count SMs: the first n_pair_items are pairs; when the pairs of a

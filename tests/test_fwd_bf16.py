@@ -244,6 +244,10 @@ def test_negative_scale(B, H, Nq, Nk, D):
     (2, 37, 256, 500, 64),    # 74 pairs: all as 148 single tiles, one round
     (1, 16, 1024, 1024, 128), # 64 pairs: 128 single tiles with 8 key tiles each
     (1, 16, 256, 256, 128),   # 16 pairs: 32 single tiles with 2 key tiles each
+    # Past the plain key limit (2048 at D = 128, 4096 at D = 64) the persistent CTAs are used
+    # only when the item list has single tiles:
+    (2, 37, 256, 3000, 128),  # 74 pairs as 148 single tiles, 24 key tiles (the last ragged)
+    (2, 37, 256, 6000, 64),   # the same at D = 64 with 47 key tiles
 ])
 def test_persistent_items_full(B, H, Nq, Nk, D):
     """Short key ranges with Nq a multiple of 256: CTAs walk several (head, tile pair) items,
