@@ -20,9 +20,10 @@
 // which most CTAs would idle), the last r pairs are listed instead as 2r
 // single items of one query tile each, provided 2r <= G: the two slots of a
 // single item run the recurrence for the same rows over alternate key tiles
-// (slot t takes tiles t, t+2, ...) and slot 0 folds slot 1's summary in with
-// the two-block formulas at the end, so the last round takes about half the
-// time of a pair round.
+// (slot t takes tiles t, t+2, ...); at the end they swap their row summaries
+// through shared memory, fold them with the two-block formulas and each writes
+// half of the head dims from both slots' O, so the last round takes about half
+// the time of a pair round.
 //
 // Roles (320 threads) as in fwd_bf16.cu's two-tile path:
 //   warp 0       TMEM allocator, then TMA producer (Q tiles per item; K_0, V_0,
@@ -33,7 +34,7 @@
 // of the slot's running key-tile count).  Per item, q_empty (Q may be
 // replaced), o_final (O complete) and o_free[t] (slot t's O has been read by
 // the epilogue, so the next item's first P V may overwrite it) complete once;
-// merge_ready (slot 1's row summaries are in shared memory) once per single
+// merge_ready (both slots' row summaries are in shared memory) once per single
 // item.
 // TMEM: S_0 [0,128) S_1 [128,256) O_0 [256,256+D) O_1 [384,384+D).
 //
